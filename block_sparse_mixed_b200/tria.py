@@ -1,0 +1,220 @@
+"""ctypes binding of libtria.so (include/tria.h), same names as the C entry points.
+
+Argument marshalling only: tensors are passed as device pointers with the
+current CUDA stream; every step of the computation runs in the library's
+kernels. torch is used for device memory and streams. If the library is
+missing this module raises at first use -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import re
+from pathlib import Path
+
+import numpy as np
+import torch
+
+_PKG = Path(__file__).resolve().parent
+LIB_PATH = _PKG / "libtria.so"
+HEADER = _PKG.parent / "include" / "tria.h"
+
+TRIA_OK, TRIA_ERR_INVALID_ARG, TRIA_ERR_UNSUPPORTED, TRIA_ERR_CUDA = 0, 1, 2, 3
+TRIA_ERR_TIMEOUT, TRIA_ERR_BOUNDS, TRIA_ERR_WORKSPACE = 4, 5, 6
+
+
+class TriaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {tria_status_string(status)} (status {status})")
+        self.status = status
+
+
+class tria_kv_cache(ctypes.Structure):
+    _fields_ = [("k8", ctypes.c_void_p), ("k4", ctypes.c_void_p), ("k8_scale", ctypes.c_void_p),
+                ("k4_scale", ctypes.c_void_p), ("v8", ctypes.c_void_p), ("v4", ctypes.c_void_p),
+                ("v8_scale", ctypes.c_void_p), ("v4_scale", ctypes.c_void_p),
+                ("B", ctypes.c_int), ("Hkv", ctypes.c_int), ("D", ctypes.c_int), ("T", ctypes.c_int),
+                ("capacity", ctypes.c_int)]
+
+
+class tria_dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("S", ctypes.c_int),
+                ("D", ctypes.c_int), ("T", ctypes.c_int)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libtria.so (raises FileNotFoundError if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not LIB_PATH.exists():
+            raise FileNotFoundError(f"{LIB_PATH} is missing: build it with python -m block_sparse_mixed_b200.build")
+        L = ctypes.CDLL(str(LIB_PATH))
+        P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+        L.tria_status_string.argtypes = [I]
+        L.tria_status_string.restype = ctypes.c_char_p
+        L.tria_cache_bytes.argtypes = [I, I, I, I, I]
+        L.tria_cache_bytes.restype = SZ
+        L.tria_cache_init.argtypes = [ctypes.POINTER(tria_kv_cache), P, SZ, I, I, I, I, I]
+        L.tria_cache_init.restype = I
+        L.tria_quantize_rows.argtypes = [P, I64, I, P, P, P, P, P]
+        L.tria_quantize_rows.restype = I
+        L.tria_quantize_kv.argtypes = [P, P, I, I, ctypes.POINTER(tria_kv_cache), P]
+        L.tria_quantize_kv.restype = I
+        L.tria_count_tiles.argtypes = [I, I, I, P]
+        L.tria_count_tiles.restype = I
+        L.tria_prefill_workspace_bytes.argtypes = [ctypes.POINTER(tria_dims)]
+        L.tria_prefill_workspace_bytes.restype = SZ
+        L.tria_prefill.argtypes = [P, ctypes.POINTER(tria_kv_cache), ctypes.POINTER(tria_dims), P, P, P, P, P,
+                                   SZ, P]
+        L.tria_prefill.restype = I
+        L.tria_decode_workspace_bytes.argtypes = [I, I, I, I, I, I]
+        L.tria_decode_workspace_bytes.restype = SZ
+        L.tria_decode.argtypes = [P, ctypes.POINTER(tria_kv_cache), P, I, P, P, P, P, P, SZ, P]
+        L.tria_decode.restype = I
+        L.tria_workspace_status.argtypes = [P, P]
+        L.tria_workspace_status.restype = I
+        _lib = L
+    return _lib
+
+
+def declared_functions() -> list[str]:
+    """Names of the functions include/tria.h declares."""
+    text = HEADER.read_text()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+[\s\*]+(tria_\w+)\s*\(", text, flags=re.M)))
+
+
+def tria_status_string(status: int) -> str:
+    return lib().tria_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int):
+    if status != TRIA_OK:
+        raise TriaError(fn, status)
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev_ptr(t: torch.Tensor) -> ctypes.c_void_p:
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("expected a contiguous CUDA tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _host_i32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+def _aligned_empty(nbytes: int, device) -> torch.Tensor:
+    """A byte buffer whose start is 256-byte aligned (torch's allocator already aligns to 512)."""
+    buf = torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+    assert buf.data_ptr() % 256 == 0
+    return buf
+
+
+class CompressedKVCache:
+    """Caller-owned compressed cache: one device buffer carved by tria_cache_init."""
+
+    def __init__(self, B: int, Hkv: int, D: int, T: int, capacity: int, device="cuda"):
+        n = lib().tria_cache_bytes(B, Hkv, D, T, capacity)
+        if n == 0:
+            raise TriaError("tria_cache_bytes", TRIA_ERR_INVALID_ARG)
+        self.buffer = _aligned_empty(n, device)
+        self.struct = tria_kv_cache()
+        _check("tria_cache_init", lib().tria_cache_init(ctypes.byref(self.struct), _dev_ptr(self.buffer), n,
+                                                         B, Hkv, D, T, capacity))
+        self.B, self.Hkv, self.D, self.T, self.capacity = B, Hkv, D, T, capacity
+
+    def plane(self, name: str) -> torch.Tensor:
+        """View of one plane: k8/v8 int8 [B,Hkv,cap,D], k4/v4 uint8 [B,Hkv,cap,D/2], *_scale fp32 [B,Hkv,cap]."""
+        base = self.buffer.data_ptr()
+        off = getattr(self.struct, name) - base
+        rows = self.B * self.Hkv * self.capacity
+        if name in ("k8", "v8"):
+            return self.buffer[off:off + rows * self.D].view(torch.int8).view(self.B, self.Hkv, self.capacity, self.D)
+        if name in ("k4", "v4"):
+            return self.buffer[off:off + rows * self.D // 2].view(self.B, self.Hkv, self.capacity, self.D // 2)
+        return self.buffer[off:off + rows * 4].view(torch.float32).view(self.B, self.Hkv, self.capacity)
+
+
+def tria_quantize_rows(X: torch.Tensor, int4: bool = True, stream=None):
+    """Codec over the rows of X (bf16 [..., D]): (c8 int8, s8 fp32, c4 uint8 packed, s4 fp32)."""
+    D = X.shape[-1]
+    rows = X.numel() // D
+    c8 = torch.empty((rows, D), dtype=torch.int8, device=X.device)
+    s8 = torch.empty(rows, dtype=torch.float32, device=X.device)
+    c4 = torch.empty((rows, D // 2), dtype=torch.uint8, device=X.device) if int4 else None
+    s4 = torch.empty(rows, dtype=torch.float32, device=X.device) if int4 else None
+    _check("tria_quantize_rows", lib().tria_quantize_rows(
+        _dev_ptr(X), rows, D, _dev_ptr(c8), _dev_ptr(s8), _dev_ptr(c4) if int4 else None,
+        _dev_ptr(s4) if int4 else None, _stream(stream)))
+    return c8, s8, c4, s4
+
+
+def tria_quantize_kv(K: torch.Tensor, V: torch.Tensor, cache: CompressedKVCache, start: int = 0, stream=None):
+    """Write K/V (bf16 [B,Hkv,S,D]) into cache positions [start, start+S)."""
+    S = K.shape[2]
+    _check("tria_quantize_kv", lib().tria_quantize_kv(_dev_ptr(K), _dev_ptr(V), S, start,
+                                                      ctypes.byref(cache.struct), _stream(stream)))
+
+
+def tria_count_tiles(nb: int, hi: int, keep: int):
+    out = np.zeros(3, np.int64)
+    _check("tria_count_tiles", lib().tria_count_tiles(nb, hi, keep, out.ctypes.data_as(ctypes.c_void_p)))
+    return tuple(int(v) for v in out)
+
+
+def tria_prefill_workspace_bytes(B, Hq, Hkv, S, D, T) -> int:
+    d = tria_dims(B, Hq, Hkv, S, D, T)
+    return int(lib().tria_prefill_workspace_bytes(ctypes.byref(d)))
+
+
+def tria_prefill(Q: torch.Tensor, cache: CompressedKVCache, hi, keep, workspace: torch.Tensor | None = None,
+                 O: torch.Tensor | None = None, LSE: torch.Tensor | None = None, stream=None):
+    """Fused prefill. Q bf16 [B,Hq,S,D]; the cache holds tokens [0,S). Returns (O bf16, LSE fp32)."""
+    B, Hq, S, D = Q.shape
+    dims = tria_dims(B, Hq, cache.Hkv, S, D, cache.T)
+    need = int(lib().tria_prefill_workspace_bytes(ctypes.byref(dims)))
+    if workspace is None:
+        workspace = _aligned_empty(need, Q.device)
+    if O is None:
+        O = torch.empty_like(Q)
+    if LSE is None:
+        LSE = torch.empty((B, Hq, S), dtype=torch.float32, device=Q.device)
+    hi_a, keep_a = _host_i32(hi), _host_i32(keep)
+    _check("tria_prefill", lib().tria_prefill(
+        _dev_ptr(Q), ctypes.byref(cache.struct), ctypes.byref(dims), hi_a.ctypes.data_as(ctypes.c_void_p),
+        keep_a.ctypes.data_as(ctypes.c_void_p), _dev_ptr(O), _dev_ptr(LSE), _dev_ptr(workspace),
+        workspace.numel(), _stream(stream)))
+    return O, LSE
+
+
+def tria_decode_workspace_bytes(B, Hq, Hkv, D, T, capacity) -> int:
+    return int(lib().tria_decode_workspace_bytes(B, Hq, Hkv, D, T, capacity))
+
+
+def tria_decode(q: torch.Tensor, cache: CompressedKVCache, kv_len, hi, keep, workspace: torch.Tensor | None = None,
+                O: torch.Tensor | None = None, LSE: torch.Tensor | None = None, stream=None):
+    """Split-KV decode. q bf16 [B,Hq,D]; kv_len host ints [B]. Returns (O bf16 [B,Hq,D], LSE fp32 [B,Hq])."""
+    B, Hq, D = q.shape
+    need = tria_decode_workspace_bytes(B, Hq, cache.Hkv, D, cache.T, cache.capacity)
+    if workspace is None:
+        workspace = _aligned_empty(need, q.device)
+    if O is None:
+        O = torch.empty_like(q)
+    if LSE is None:
+        LSE = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    kv, hi_a, keep_a = _host_i32(kv_len), _host_i32(hi), _host_i32(keep)
+    _check("tria_decode", lib().tria_decode(
+        _dev_ptr(q), ctypes.byref(cache.struct), kv.ctypes.data_as(ctypes.c_void_p), Hq,
+        hi_a.ctypes.data_as(ctypes.c_void_p), keep_a.ctypes.data_as(ctypes.c_void_p), _dev_ptr(O), _dev_ptr(LSE),
+        _dev_ptr(workspace), workspace.numel(), _stream(stream)))
+    return O, LSE
+
+
+def tria_workspace_status(workspace: torch.Tensor, stream=None) -> int:
+    return int(lib().tria_workspace_status(_dev_ptr(workspace), _stream(stream)))

@@ -1,0 +1,156 @@
+/*
+ * tria.h -- C ABI of the block-sparse mixed-precision causal attention library
+ * (TriAttention-style), built for NVIDIA B200 (sm_100a).
+ *
+ * What is computed. Attention is cut into tiles of T query tokens x T key
+ * tokens. Each tile of query block i and key block j (j <= i) gets one of three
+ * actions -- skip, compute with 4-bit codes, compute with 8-bit codes -- from its
+ * distance d = i - j to the diagonal and a per-head pair of boundaries
+ * (hi, keep): 8-bit if d < hi, 4-bit if hi <= d < keep, skipped if d >= keep.
+ * Key block 0 and the diagonal block are always computed with 8-bit codes.
+ * (rit.work TriAttention page, section "Какие связи можно не считать, а какие
+ * нельзя удалять", paragraphs three to five; the half-open bands and the
+ * per-query-head pair are readings of that text.) All kept tiles of a query row
+ * are reduced into one normalised softmax result, and the prepared K/V go to a
+ * compressed KV cache that decode reads (section "Как калибровка распределяет
+ * вычисления между головами", last paragraph).
+ *
+ * Codec (a reading; the page names only 4 and 8 bits): per token and per plane,
+ * s = max|x| / 127 (int8) or max|x| / 7 (int4) in fp32 with IEEE division,
+ * code = rint(x / s) with ties to even, clamped to [-127,127] / [-7,7]; an
+ * all-zero row has scale 0 and codes 0. The tile's plane applies to Q, K and V.
+ * Scores are (integer code dot product) * s_q * s_k / sqrt(D); softmax in fp32;
+ * P.V in bf16 with fp32 accumulation. GQA maps query head h to KV head
+ * h / (Hq / Hkv) (llmis.ru chapter 3.5, section 4).
+ *
+ * Conventions for every call:
+ *  - Pointers named "device" are CUDA device pointers; "host" are host memory.
+ *  - bf16 tensors are contiguous, row-major, [B, H, tokens, D] ("BHSD").
+ *  - Device pointers must be 16-byte aligned; the workspace 256-byte aligned.
+ *  - All memory is owned by the caller; the library allocates nothing.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*,
+ *    NULL = legacy default stream) and return a tria_status at once. Argument
+ *    errors are found on the host before any launch and leave memory untouched.
+ *  - Supported: D in {64, 128}, T in {64, 128}, Hq % Hkv == 0, Hq/Hkv <= 16,
+ *    Hq <= 256, B <= 1024, device compute capability 10.0 (sm_100a).
+ *  - Kernels never trap. A pipeline wait that runs past its limit, or an index
+ *    that fails its check, sets an error word in the workspace and the kernel
+ *    returns; tria_workspace_status() reports it.
+ */
+#ifndef TRIA_H_
+#define TRIA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TRIA_OK = 0,
+  TRIA_ERR_INVALID_ARG = 1,   /* bad shape, pointer, alignment or policy */
+  TRIA_ERR_UNSUPPORTED = 2,   /* D, T, head ratio or GPU not supported */
+  TRIA_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed */
+  TRIA_ERR_TIMEOUT = 4,       /* a device-side pipeline wait ran past its limit */
+  TRIA_ERR_BOUNDS = 5,        /* a device-side index check failed */
+  TRIA_ERR_WORKSPACE = 6      /* workspace missing or smaller than required */
+} tria_status;
+
+/* Compressed KV cache: the "prepared K and V" of the method, one row per token.
+ * For X in {k, v}:
+ *   x8        int8  [B, Hkv, capacity, D]      8-bit codes
+ *   x4        uint8 [B, Hkv, capacity, D/2]    4-bit codes, two per byte:
+ *                                              element 2m in the low nibble,
+ *                                              element 2m+1 in the high nibble,
+ *                                              4-bit two's complement
+ *   x8_scale  fp32  [B, Hkv, capacity]         per-token scale of the 8-bit plane
+ *   x4_scale  fp32  [B, Hkv, capacity]         per-token scale of the 4-bit plane
+ * All eight pointers are device pointers, 16-byte aligned. capacity is a
+ * multiple of T. The struct itself is host memory, read during the call only. */
+typedef struct {
+  int8_t* k8;
+  uint8_t* k4;
+  float* k8_scale;
+  float* k4_scale;
+  int8_t* v8;
+  uint8_t* v4;
+  float* v8_scale;
+  float* v4_scale;
+  int B, Hkv, D, T, capacity;
+} tria_kv_cache;
+
+/* Shape of a prefill: B sequences of S tokens, Hq query heads, Hkv KV heads. */
+typedef struct {
+  int B, Hq, Hkv, S, D, T;
+} tria_dims;
+
+/* Human-readable name of a status code (static string). */
+const char* tria_status_string(int status);
+
+/* Bytes needed to hold every plane of a cache carved by tria_cache_init. */
+size_t tria_cache_bytes(int B, int Hkv, int D, int T, int capacity);
+
+/* Fill `cache` with plane pointers carved from one caller buffer `base`
+ * (device, 256-byte aligned, at least tria_cache_bytes(...) bytes). Writes no
+ * device memory. Returns TRIA_ERR_INVALID_ARG on a bad shape or alignment. */
+int tria_cache_init(tria_kv_cache* cache, void* base, size_t bytes,
+                    int B, int Hkv, int D, int T, int capacity);
+
+/* Codec over arbitrary rows (used for Q and by the tests).
+ * X: device bf16 [rows, D]. Outputs (device): c8 int8 [rows, D], s8 fp32
+ * [rows], c4 uint8 [rows, D/2] packed as in the cache, s4 fp32 [rows].
+ * Any of c4/s4 may be NULL to skip that plane. Bit-exact with the codec rule
+ * above. */
+int tria_quantize_rows(const void* X, int64_t rows, int D, int8_t* c8, float* s8,
+                       uint8_t* c4, float* s4, void* stream);
+
+/* Write the prepared K/V of S tokens into cache positions [start, start+S).
+ * K, V: device bf16 [B, Hkv, S, D] (B, Hkv, D as in the cache).
+ * Requires 0 <= start, start + S <= capacity, S >= 1. Any start is allowed, so
+ * this also appends decode tokens one at a time (S = 1). */
+int tria_quantize_kv(const void* K, const void* V, int S, int start,
+                     const tria_kv_cache* cache, void* stream);
+
+/* Tile counts of one head over nb x nb blocks (host-only helper):
+ * out[0] = int8 tiles, out[1] = int4 tiles, out[2] = skipped causal tiles. */
+int tria_count_tiles(int nb, int hi, int keep, int64_t* out);
+
+/* Workspace bytes tria_prefill needs for `dims` (0 if dims are invalid). */
+size_t tria_prefill_workspace_bytes(const tria_dims* dims);
+
+/* Fused block-sparse mixed-precision causal prefill.
+ * Q: device bf16 [B, Hq, S, D]; cache: holds K/V tokens [0, S) (written by
+ * tria_quantize_kv); hi, keep: HOST int32 arrays of length Hq with
+ * 0 <= hi <= keep (keep may exceed the block count). S % T == 0,
+ * S <= capacity. O: device bf16 [B, Hq, S, D]; LSE: device fp32 [B, Hq, S],
+ * natural log-sum-exp of the row's kept scaled scores. workspace: device,
+ * 256-byte aligned, >= tria_prefill_workspace_bytes(dims). */
+int tria_prefill(const void* Q, const tria_kv_cache* cache, const tria_dims* dims,
+                 const int32_t* hi, const int32_t* keep, void* O, float* LSE,
+                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes tria_decode needs (0 if the arguments are invalid). */
+size_t tria_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int T, int capacity);
+
+/* Split-KV decode of one new token per sequence over the compressed cache.
+ * q: device bf16 [B, Hq, D]; kv_len: HOST int32 [B], 1 <= kv_len[b] <=
+ * capacity: the token sits at position kv_len[b]-1 and is already in the
+ * cache, so its block is the diagonal block. hi, keep: HOST int32 [Hq].
+ * O: device bf16 [B, Hq, D]; LSE: device fp32 [B, Hq]. Only the kept blocks
+ * of the planes some head of a KV group needs are read; partial results of
+ * the splits are merged by log-sum-exp. */
+int tria_decode(const void* q, const tria_kv_cache* cache, const int32_t* kv_len, int Hq,
+                const int32_t* hi, const int32_t* keep, void* O, float* LSE,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronise `stream` and return the device-side error word of `workspace`
+ * (TRIA_OK, TRIA_ERR_TIMEOUT or TRIA_ERR_BOUNDS); the word is cleared by
+ * every tria_prefill / tria_decode call that uses this workspace. */
+int tria_workspace_status(const void* workspace, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TRIA_H_ */

@@ -1,0 +1,117 @@
+"""C-ABI boundary checks that need no GPU: the library loads, exports every
+function include/tria.h declares, and its host-side logic (sizes, cache
+carving, tile counting, argument validation) behaves as documented."""
+import ctypes
+
+import numpy as np
+import pytest
+
+from block_sparse_mixed_b200 import tria
+from block_sparse_mixed_b200.build import build
+
+
+@pytest.fixture(scope="module")
+def L():
+    build()
+    return tria.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = tria.declared_functions()
+    assert len(names) == 11, names
+    for n in ("tria_quantize_kv", "tria_prefill", "tria_decode", "tria_quantize_rows"):
+        assert n in names
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in tria.h but not exported"
+
+
+def test_status_strings(L):
+    for s in range(7):
+        assert tria.tria_status_string(s)
+    assert tria.tria_status_string(0) == "ok"
+
+
+def test_cache_sizes_and_carving(L):
+    B, Hkv, D, T, cap = 2, 3, 128, 64, 256
+    n = L.tria_cache_bytes(B, Hkv, D, T, cap)
+    rows = B * Hkv * cap
+    assert n >= 2 * (rows * D + rows * D // 2 + 2 * rows * 4)
+    assert L.tria_cache_bytes(B, Hkv, 96, T, cap) == 0          # unsupported D
+    assert L.tria_cache_bytes(B, Hkv, D, T, cap + 1) == 0       # capacity not a multiple of T
+    c = tria.tria_kv_cache()
+    base = 1 << 40                                             # never dereferenced
+    assert L.tria_cache_init(ctypes.byref(c), ctypes.c_void_p(base), n, B, Hkv, D, T, cap) == 0
+    ptrs = [c.k8, c.k4, c.k8_scale, c.k4_scale, c.v8, c.v4, c.v8_scale, c.v4_scale]
+    assert ptrs[0] == base and all(p % 256 == 0 for p in ptrs)
+    sizes = [rows * D, rows * D // 2, rows * 4, rows * 4] * 2
+    for p, q, s in zip(ptrs, ptrs[1:], sizes):
+        assert q - p >= s                                      # planes do not overlap
+    assert ptrs[-1] + rows * 4 <= base + n
+    assert L.tria_cache_init(ctypes.byref(c), ctypes.c_void_p(base + 16), n, B, Hkv, D, T, cap) == 1
+    assert L.tria_cache_init(ctypes.byref(c), ctypes.c_void_p(base), n - 1, B, Hkv, D, T, cap) == 1
+
+
+def test_tile_counts_match_oracle(L, oracle_mod):
+    for nb in (1, 2, 7, 16, 33):
+        for hi in range(0, 6):
+            for keep in range(hi, hi + 8):
+                assert tria.tria_count_tiles(nb, hi, keep) == oracle_mod.action_counts(nb, hi, keep)
+    with pytest.raises(tria.TriaError):
+        tria.tria_count_tiles(8, 3, 2)
+
+
+def test_workspace_sizes(L):
+    assert tria.tria_prefill_workspace_bytes(1, 32, 8, 8192, 128, 64) > 0
+    assert tria.tria_prefill_workspace_bytes(1, 32, 8, 8192 + 1, 128, 64) == 0   # S % T
+    assert tria.tria_prefill_workspace_bytes(1, 30, 8, 8192, 128, 64) == 0       # Hq % Hkv
+    assert tria.tria_prefill_workspace_bytes(1, 32, 8, 8192, 80, 64) == 0        # D
+    assert tria.tria_decode_workspace_bytes(64, 32, 8, 128, 128, 32768) > 0
+    assert tria.tria_decode_workspace_bytes(64, 64, 2, 128, 128, 32768) == 0     # 32 heads per group
+
+
+def _fake_cache(B=1, Hkv=2, D=128, T=64, cap=512):
+    c = tria.tria_kv_cache()
+    n = tria.lib().tria_cache_bytes(B, Hkv, D, T, cap)
+    assert tria.lib().tria_cache_init(ctypes.byref(c), ctypes.c_void_p(1 << 40), n, B, Hkv, D, T, cap) == 0
+    return c
+
+
+def test_host_validation_rejects_bad_arguments(L):
+    fake = ctypes.c_void_p(1 << 41)
+    c = _fake_cache()
+    i32 = lambda v: np.ascontiguousarray(v, np.int32)
+    hi, keep = i32([1, 2, 1, 2]), i32([3, 5, 3, 5])
+    P = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    ws = ctypes.c_void_p(1 << 42)
+    # quantize_kv: start + S beyond capacity, null pointers
+    assert L.tria_quantize_kv(fake, fake, 600, 0, ctypes.byref(c), None) == tria.TRIA_ERR_INVALID_ARG
+    assert L.tria_quantize_kv(None, fake, 10, 0, ctypes.byref(c), None) == tria.TRIA_ERR_INVALID_ARG
+    assert L.tria_quantize_kv(fake, fake, 10, -1, ctypes.byref(c), None) == tria.TRIA_ERR_INVALID_ARG
+    # prefill: S % T, keep < hi, negative hi, unsupported D, workspace too small
+    d = tria.tria_dims(1, 4, 2, 500, 128, 64)
+    assert L.tria_prefill(fake, ctypes.byref(c), ctypes.byref(d), P(hi), P(keep), fake, fake, ws, 1 << 40,
+                          None) == tria.TRIA_ERR_INVALID_ARG
+    d = tria.tria_dims(1, 4, 2, 512, 128, 64)
+    assert L.tria_prefill(fake, ctypes.byref(c), ctypes.byref(d), P(i32([2, 2, 2, 2])), P(i32([1, 5, 5, 5])),
+                          fake, fake, ws, 1 << 40, None) == tria.TRIA_ERR_INVALID_ARG
+    assert L.tria_prefill(fake, ctypes.byref(c), ctypes.byref(d), P(i32([-1, 2, 2, 2])), P(keep),
+                          fake, fake, ws, 1 << 40, None) == tria.TRIA_ERR_INVALID_ARG
+    assert L.tria_prefill(fake, ctypes.byref(c), ctypes.byref(d), P(hi), P(keep), fake, fake, ws, 16,
+                          None) == tria.TRIA_ERR_WORKSPACE
+    d96 = tria.tria_dims(1, 4, 2, 512, 96, 64)
+    assert L.tria_prefill(fake, ctypes.byref(c), ctypes.byref(d96), P(hi), P(keep), fake, fake, ws, 1 << 40,
+                          None) == tria.TRIA_ERR_UNSUPPORTED
+    big = tria.tria_dims(1, 4, 2, 1024, 128, 64)          # S beyond the cache capacity
+    assert L.tria_prefill(fake, ctypes.byref(c), ctypes.byref(big), P(hi), P(keep), fake, fake, ws, 1 << 40,
+                          None) == tria.TRIA_ERR_INVALID_ARG
+    # decode: kv_len out of range, head ratio
+    assert L.tria_decode(fake, ctypes.byref(c), P(i32([513])), 4, P(hi), P(keep), fake, fake, ws, 1 << 40,
+                         None) == tria.TRIA_ERR_INVALID_ARG
+    assert L.tria_decode(fake, ctypes.byref(c), P(i32([0])), 4, P(hi), P(keep), fake, fake, ws, 1 << 40,
+                         None) == tria.TRIA_ERR_INVALID_ARG
+    assert L.tria_decode(fake, ctypes.byref(c), P(i32([10])), 3, P(hi), P(keep), fake, fake, ws, 1 << 40,
+                         None) == tria.TRIA_ERR_INVALID_ARG
+    # codec: unsupported width, unaligned pointer
+    assert L.tria_quantize_rows(fake, 4, 96, fake, fake, fake, fake, None) == tria.TRIA_ERR_UNSUPPORTED
+    assert L.tria_quantize_rows(ctypes.c_void_p((1 << 41) + 2), 4, 128, fake, fake, fake, fake,
+                                None) == tria.TRIA_ERR_INVALID_ARG

@@ -1,0 +1,216 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Every input is seeded and synthetic (block_sparse_mixed_b200.workloads); the
+oracle never sees anything the GPU computed. Codes and scales must match bit
+for bit; O and LSE within the tolerances in tests/parity.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_mixed_b200 import workloads as W
+from parity import compare_lse, compare_o, rows_of
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def T():
+    from block_sparse_mixed_b200.build import build
+    build()
+    from block_sparse_mixed_b200 import tria
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return tria
+
+
+def seeded(shape, seed, device="cpu", scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(shape, generator=g) * scale).to(torch.bfloat16).to(device)
+
+
+# ---------------------------------------------------------------- codec
+
+def test_codec_bit_exact(T, oracle_mod):
+    for D in (64, 128):
+        x = seeded((4099, D), 100 + D)
+        x[0] = 0                                    # zero row
+        x[1] = (x[1].float() * 1e-30).to(torch.bfloat16)   # tiny magnitudes
+        x[2] = -x[2].abs()
+        x[3, :8] = torch.tensor([127, 45.5, -37.5, 0.5, -0.5, 1.5, 2.5, -2.5])   # exact ties (s8 = 1)
+        x[3, 8:] = 0
+        x[4, :8] = torch.tensor([7, 4.5, 2.5, -0.5, 1.5, -5.5, 6.5, 0.25])       # exact ties (s4 = 1)
+        x[4, 8:] = 0
+        c8, s8, c4, s4 = T.tria_quantize_rows(x.cuda())
+        r8, rs8, r4, rs4 = oracle_mod.quantize_rows(x, D)
+        assert np.array_equal(c8.cpu().numpy(), r8)
+        assert np.array_equal(s8.cpu().numpy().view(np.uint32), rs8.view(np.uint32))
+        assert np.array_equal(s4.cpu().numpy().view(np.uint32), rs4.view(np.uint32))
+        assert np.array_equal(c4.cpu().numpy(), oracle_mod.pack_int4(r4))
+
+
+def test_cache_write_and_append_bit_exact(T, oracle_mod):
+    B, Hkv, D, Tb, cap = 2, 3, 128, 64, 320
+    cache = T.CompressedKVCache(B, Hkv, D, Tb, cap)
+    cache.buffer.fill_(0x5A)
+    K, V = seeded((B, Hkv, 200, D), 7), seeded((B, Hkv, 200, D), 8)
+    T.tria_quantize_kv(K.cuda(), V.cuda(), cache, start=0)
+    k1, v1 = seeded((B, Hkv, 1, D), 9), seeded((B, Hkv, 1, D), 10)
+    T.tria_quantize_kv(k1.cuda(), v1.cuda(), cache, start=200)          # one-token append
+    torch.cuda.synchronize()
+    Kall, Vall = torch.cat([K, k1], 2), torch.cat([V, v1], 2)
+    for X, p in ((Kall, "k"), (Vall, "v")):
+        r8, rs8, r4, rs4 = oracle_mod.quantize_rows(X, D)
+        r8 = r8.reshape(B, Hkv, 201, D)
+        r4p = oracle_mod.pack_int4(r4).reshape(B, Hkv, 201, D // 2)
+        assert np.array_equal(cache.plane(p + "8")[:, :, :201].cpu().numpy(), r8)
+        assert np.array_equal(cache.plane(p + "4")[:, :, :201].cpu().numpy(), r4p)
+        assert np.array_equal(cache.plane(p + "8_scale")[:, :, :201].cpu().numpy().reshape(-1).view(np.uint32),
+                              rs8.view(np.uint32))
+        assert np.array_equal(cache.plane(p + "4_scale")[:, :, :201].cpu().numpy().reshape(-1).view(np.uint32),
+                              rs4.view(np.uint32))
+        assert (cache.plane(p + "8")[:, :, 201:].cpu().view(torch.uint8) == 0x5A).all()  # untouched
+
+
+# ---------------------------------------------------------------- prefill
+
+def run_prefill(T, Q, K, V, Tb, hi, keep, cap=None):
+    B, Hq, S, D = Q.shape
+    Hkv = K.shape[1]
+    cache = T.CompressedKVCache(B, Hkv, D, Tb, cap or S)
+    T.tria_quantize_kv(K.cuda(), V.cuda(), cache)
+    ws = torch.empty(T.tria_prefill_workspace_bytes(B, Hq, Hkv, S, D, Tb), dtype=torch.uint8, device="cuda")
+    O, L = T.tria_prefill(Q.cuda(), cache, hi, keep, workspace=ws)
+    torch.cuda.synchronize()
+    assert T.tria_workspace_status(ws) == 0
+    return O, L, cache
+
+
+PREFILL_CASES = {
+    # name: (B, Hq, Hkv, S, D, T, policies)
+    "tiny_512_d64_t64": (1, 2, 2, 512, 64, 64, [(1, 3), (2, 5)]),
+    "gqa_t128_d128": (1, 4, 1, 1280, 128, 128, [(1, 3), (2, 6), (0, 2), (4, 4)]),
+    "ragged_tile_t64": (2, 4, 2, 576, 128, 64, [(1, 2), (3, 9), (0, 0), (2, 4)]),
+    "d64_t128": (1, 2, 1, 768, 64, 128, [(2, 3), (1, 6)]),
+    "protected_only": (1, 2, 2, 640, 128, 64, [(0, 0), (0, 1)]),
+    "dense_int8": (1, 2, 1, 512, 128, 128, [(4, 4), (9, 9)]),
+    "all_int4_band": (1, 2, 1, 512, 128, 64, [(0, 20), (1, 20)]),
+}
+
+
+@pytest.mark.parametrize("name", list(PREFILL_CASES))
+def test_prefill_matches_oracle(T, oracle_mod, name):
+    B, Hq, Hkv, S, D, Tb, pol = PREFILL_CASES[name]
+    hi = np.array([p[0] for p in pol], np.int32)
+    keep = np.array([p[1] for p in pol], np.int32)
+    seed = sum(map(ord, name))
+    Q, K, V = seeded((B, Hq, S, D), seed), seeded((B, Hkv, S, D), seed + 1), seeded((B, Hkv, S, D), seed + 2)
+    O, L, _ = run_prefill(T, Q, K, V, Tb, hi, keep)
+    O_ref, L_ref = oracle_mod.prefill_rows(Q, K, V, Tb, hi, keep)
+    compare_o(O, O_ref.reshape(B, Hq, S, D), name)
+    compare_lse(L, L_ref.reshape(B, Hq, S), name)
+
+
+def test_prefill_tiny_workload(T, oracle_mod):
+    w = W.WORKLOADS["tiny_prefill"]
+    Q, K, V = W.prefill_inputs(w)
+    hi, keep = W.policy(w)
+    O, L, _ = run_prefill(T, Q, K, V, w.T, hi, keep)
+    O_ref, L_ref = oracle_mod.prefill_rows(Q, K, V, w.T, hi, keep)
+    compare_o(O, O_ref.reshape(O.shape), "tiny")
+    compare_lse(L, L_ref.reshape(L.shape), "tiny")
+
+
+def test_prefill_llama_workload_sampled_rows(T, oracle_mod):
+    """Full-size 8192-token GQA workload; the oracle checks sampled rows."""
+    w = W.WORKLOADS["llama_prefill"]
+    Q, K, V = W.prefill_inputs(w)
+    hi, keep = W.policy(w)
+    O, L, _ = run_prefill(T, Q, K, V, w.T, hi, keep)
+    rng = np.random.RandomState(0)
+    picks = [(0, h, t) for h in range(w.Hq) for t in (0, 63, 64, w.S - 1)]
+    picks += [(0, int(rng.randint(w.Hq)), int(rng.randint(w.S))) for _ in range(256)]
+    rows = rows_of(w.B, w.Hq, w.S, picks)
+    O_ref, L_ref = oracle_mod.prefill_rows(Q, K, V, w.T, hi, keep, rows=rows)
+    idx = torch.from_numpy(rows)
+    compare_o(O.reshape(-1, w.D).cpu()[idx], O_ref, "llama sampled")
+    compare_lse(L.reshape(-1).cpu()[idx], L_ref, "llama sampled")
+
+
+def test_prefill_skipped_blocks_are_never_read(T, oracle_mod):
+    """Overwrite the cache codes of one key block: rows whose tile with it is
+    skipped must come out bit-identical; rows that keep it must change."""
+    B, Hq, Hkv, S, D, Tb = 1, 2, 1, 1024, 128, 64
+    hi = np.array([1, 2], np.int32)
+    keep = np.array([3, 5], np.int32)
+    Q, K, V = seeded((B, Hq, S, D), 61), seeded((B, Hkv, S, D), 62), seeded((B, Hkv, S, D), 63)
+    O1, L1, cache = run_prefill(T, Q, K, V, Tb, hi, keep)
+    j0 = 4
+    K2, V2 = K.clone(), V.clone()
+    K2[:, :, j0 * Tb:(j0 + 1) * Tb] = seeded((B, Hkv, Tb, D), 64, scale=3.0)
+    V2[:, :, j0 * Tb:(j0 + 1) * Tb] = seeded((B, Hkv, Tb, D), 65, scale=3.0)
+    O2, L2, _ = run_prefill(T, Q, K2, V2, Tb, hi, keep)
+    nb = S // Tb
+    for h in range(Hq):
+        amap = oracle_mod.action_map(nb, int(hi[h]), int(keep[h]))
+        for i in range(nb):
+            same = torch.equal(O1[0, h, i * Tb:(i + 1) * Tb], O2[0, h, i * Tb:(i + 1) * Tb])
+            assert same == (amap[i, j0] not in (4, 8)), (h, i, amap[i, j0])
+
+
+# ---------------------------------------------------------------- decode
+
+DECODE_CASES = {
+    # name: (B, Hq, Hkv, D, T, cap, kv_len, policies per head)
+    "t128_ragged": (3, 8, 2, 128, 128, 2048, [2048, 1000, 129],
+                    [(4, 9), (1, 3), (0, 0), (2, 16), (6, 6), (1, 2), (3, 7), (0, 5)]),
+    "t64_d64": (2, 4, 1, 64, 64, 640, [640, 65], [(1, 3), (2, 9), (0, 1), (3, 4)]),
+    "single_block": (2, 2, 2, 128, 128, 256, [1, 128], [(1, 4), (0, 2)]),
+    "g16": (1, 16, 1, 128, 64, 1024, [777], [(h % 4, 2 + h) for h in range(16)]),
+}
+
+
+def run_decode(T, q, K, V, Tb, kv_len, hi, keep):
+    B, Hkv, cap, D = K.shape
+    cache = T.CompressedKVCache(B, Hkv, D, Tb, cap)
+    T.tria_quantize_kv(K.cuda(), V.cuda(), cache)
+    O, L = T.tria_decode(q.cuda(), cache, kv_len, hi, keep)
+    torch.cuda.synchronize()
+    return O, L
+
+
+@pytest.mark.parametrize("name", list(DECODE_CASES))
+def test_decode_matches_oracle(T, oracle_mod, name):
+    B, Hq, Hkv, D, Tb, cap, kv_len, pol = DECODE_CASES[name]
+    hi = np.array([p[0] for p in pol], np.int32)
+    keep = np.array([p[1] for p in pol], np.int32)
+    seed = sum(map(ord, name))
+    q, K, V = seeded((B, Hq, D), seed), seeded((B, Hkv, cap, D), seed + 1), seeded((B, Hkv, cap, D), seed + 2)
+    kv = np.array(kv_len, np.int32)
+    O, L = run_decode(T, q, K, V, Tb, kv, hi, keep)
+    O_ref, L_ref = oracle_mod.decode(q, K, V, Tb, kv, hi, keep)
+    compare_o(O, O_ref, name)
+    compare_lse(L, L_ref, name)
+
+
+def test_decode_workload_four_sequences(T, oracle_mod):
+    """The 32768-token decode workload's shapes and policy, 4 of its 64 sequences."""
+    w = W.scaled(W.WORKLOADS["decode"], B=4)
+    q, K, V, kv = W.decode_inputs(w)
+    hi, keep = W.policy(w)
+    O, L = run_decode(T, q, K, V, w.T, kv, hi, keep)
+    O_ref, L_ref = oracle_mod.decode(q, K, V, w.T, kv, hi, keep)
+    compare_o(O, O_ref, "decode workload")
+    compare_lse(L, L_ref, "decode workload")
+
+
+def test_decode_equals_last_prefill_row(T):
+    """Same cache, same policy: decode of token S-1 reproduces prefill row S-1."""
+    B, Hq, Hkv, S, D, Tb = 2, 4, 1, 1024, 128, 128
+    hi = np.array([1, 2, 0, 3], np.int32)
+    keep = np.array([3, 4, 5, 3], np.int32)
+    Q, K, V = seeded((B, Hq, S, D), 71), seeded((B, Hkv, S, D), 72), seeded((B, Hkv, S, D), 73)
+    O, L, cache = run_prefill(T, Q, K, V, Tb, hi, keep)
+    Od, Ld = T.tria_decode(Q[:, :, S - 1].contiguous().cuda(), cache, np.full(B, S, np.int32), hi, keep)
+    torch.cuda.synchronize()
+    assert (Od.float() - O[:, :, S - 1].float()).abs().max().item() <= 1e-2
+    assert (Ld - L[:, :, S - 1]).abs().max().item() <= 1e-3
