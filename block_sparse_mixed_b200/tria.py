@@ -218,3 +218,26 @@ def tria_decode(q: torch.Tensor, cache: CompressedKVCache, kv_len, hi, keep, wor
 
 def tria_workspace_status(workspace: torch.Tensor, stream=None) -> int:
     return int(lib().tria_workspace_status(_dev_ptr(workspace), _stream(stream)))
+
+
+def tria_decode_static(q: torch.Tensor, cache: CompressedKVCache, kv_len, hi, keep, O: torch.Tensor | None = None,
+                       LSE: torch.Tensor | None = None, stream=None):
+    """tria_decode with the library's fixed device scratch instead of a caller workspace
+    (for callers that cannot allocate device memory; see include/tria.h)."""
+    L = lib()
+    if not getattr(L.tria_decode_static, "_typed", False):
+        P = ctypes.c_void_p
+        L.tria_decode_static.argtypes = [P, ctypes.POINTER(tria_kv_cache), P, ctypes.c_int, P, P, P, P, P]
+        L.tria_decode_static.restype = ctypes.c_int
+        L.tria_decode_static._typed = True
+    B, Hq, D = q.shape
+    if O is None:
+        O = torch.empty_like(q)
+    if LSE is None:
+        LSE = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    kv, hi_a, keep_a = _host_i32(kv_len), _host_i32(hi), _host_i32(keep)
+    _check("tria_decode_static", L.tria_decode_static(
+        _dev_ptr(q), ctypes.byref(cache.struct), kv.ctypes.data_as(ctypes.c_void_p), Hq,
+        hi_a.ctypes.data_as(ctypes.c_void_p), keep_a.ctypes.data_as(ctypes.c_void_p), _dev_ptr(O), _dev_ptr(LSE),
+        _stream(stream)))
+    return O, LSE

@@ -144,6 +144,28 @@ int tria_decode(const void* q, const tria_kv_cache* cache, const int32_t* kv_len
                 const int32_t* hi, const int32_t* keep, void* O, float* LSE,
                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* Bytes of the fixed device scratch array used by tria_decode_static. */
+#define TRIA_DECODE_STATIC_SCRATCH_BYTES (40u << 20)
+
+/* Split-KV decode without a caller workspace and without allocating.
+ * No counterpart in the paper: this is a deployment convenience for callers
+ * that cannot allocate device memory -- for example a plugin inside a host
+ * application whose device memory is fully budgeted in advance, or a
+ * latency-critical loop that must not call cudaMalloc, which may synchronise
+ * the device. Arguments and results are those of tria_decode minus the
+ * workspace. The scratch is one fixed __device__ array of
+ * TRIA_DECODE_STATIC_SCRATCH_BYTES (40 MiB) inside this library, held by every
+ * GPU that loads it until the process exits. Problems whose decode workspace
+ * (tria_decode_workspace_bytes) is larger are rejected with
+ * TRIA_ERR_WORKSPACE before anything runs. The first call on each device looks
+ * up the array's device address (cudaGetSymbolAddress) with that device
+ * current; make that first call before any stream capture. All calls on a
+ * device share the array: each call clears what must start at zero, and calls
+ * whose GPU work overlaps (unordered streams) race on it. Device-side pipeline
+ * errors land in the shared array's error word and are not reported here. */
+int tria_decode_static(const void* q, const tria_kv_cache* cache, const int32_t* kv_len, int Hq,
+                       const int32_t* hi, const int32_t* keep, void* O, float* LSE, void* stream);
+
 /* Synchronise `stream` and return the device-side error word of `workspace`
  * (TRIA_OK, TRIA_ERR_TIMEOUT or TRIA_ERR_BOUNDS); the word is cleared by
  * every tria_prefill / tria_decode call that uses this workspace. */
