@@ -380,8 +380,11 @@ def main():
     ap.add_argument("--workload", default="llama_prefill", choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (smaller profiling cases)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    if args.batch > 0:
+        W.WORKLOADS[args.workload] = W.scaled(W.WORKLOADS[args.workload], B=args.batch)
     w = W.WORKLOADS[args.workload]
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
