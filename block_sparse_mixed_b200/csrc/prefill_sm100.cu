@@ -11,18 +11,25 @@
 // How. A persistent CTA owns one 128-row query tile at a time (one query block
 // of T = 128, or two query blocks of T = 64) of one (batch, query head). The
 // key blocks the tile keeps are walked in ascending order; a key block whose
-// rows need both planes is loaded once per plane. Warp roles:
-//   warps 0-3  softmax: one TMEM lane (query row) per thread;
-//   warp 4     producer: TMA loads of Q codes, K codes, V tiles and K scales,
-//              only for kept (block, plane) pairs;
-//   warp 5     MMA issuer: S = Q.K^T on tcgen05 kind::i8 (int32 in TMEM), then
-//              O += P.V on tcgen05 kind::f16 (bf16 P read from TMEM, fp32 O in TMEM).
-// S is double-buffered in TMEM so QK of load g+1 overlaps the softmax of load g.
+// rows need both planes is loaded once per plane ("load" below = one kept
+// (key block, plane) pair). Warp roles:
+//   warps 0-15  softmax, as two "pairs" of warpgroups that take the loads in
+//               turn (ping-pong: pair p handles loads of parity p, using S slot p
+//               and O accumulator p in TMEM). Inside a pair, warpgroup `half`
+//               takes keys [half*T/2, (half+1)*T/2) of every row; the two halves
+//               of a row agree on its maximum through shared memory and a named
+//               barrier. Four softmax warps per SM sub-partition hide latency.
+//   warp 16     producer: TMA loads of Q codes, K codes, V tiles and K scales,
+//               only for kept (block, plane) pairs;
+//   warp 17     MMA issuer: S = Q.K^T on tcgen05 kind::i8 (int32 in TMEM), then
+//               O += P.V on tcgen05 kind::f16 (bf16 P read from TMEM, fp32 O in TMEM).
+//   warps 18-19 only take part in the register hand-over.
 // The softmax dequantises S with the row's Q scale and the key's K scale,
-// applies the causal mask on the diagonal block, keeps a running maximum that
-// is only raised when it grows by more than 2^8 (so O is rarely rescaled),
-// writes P as bf16 over the S columns, and finally normalises O.
-// Rows whose own tile action differs from the load's plane write P = 0.
+// masks the diagonal block causally, keeps a running maximum that is only
+// raised when it grows by more than 2^8 (so O is rarely rescaled), and writes P
+// as bf16 over the S columns. Rows whose own tile action differs from the
+// load's plane write P = 0. The two accumulators of a row are merged and
+// normalised in the tile epilogue.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -34,14 +41,24 @@
 namespace tria {
 namespace {
 
-constexpr int kRows = 128;             // query rows per tile (tcgen05 M)
-constexpr int kThreads = 192;          // 4 softmax warps + producer warp + MMA warp
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kSlots = 2;              // S buffers in TMEM
+constexpr int kRows = 128;              // query rows per tile (tcgen05 M)
+constexpr int kThreads = 640;           // 20 warps
+constexpr int kSoftmaxWarps = 16;
+constexpr int kPairThreads = 256;       // softmax threads of one pair (P arrivals per load)
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;
+// Register split (setmaxnreg): launched at 96 per thread (640 x 96 = 61,440; five
+// warps per sub-partition x 32 x 96 = 15,360 of its 16,384); the four softmax
+// warpgroups rise to 104 and the producer/MMA warpgroup drops to 64:
+// 4 x 128 x 104 + 128 x 64 = 61,440, within the launch total.
+constexpr int kRegsSoftmax = 104;
+constexpr int kRegsOther = 64;
+constexpr int kSlots = 2;               // S buffers in TMEM, one per pair
 constexpr int kTmemCols = 512;
-constexpr int kOCol = 256;             // O accumulator columns [256, 256 + D)
-constexpr float kRescaleLog2 = 8.0f;   // raise the running max only past this growth
+constexpr float kRescaleLog2 = 8.0f;    // raise the running max only past this growth
+
+// O accumulator of pair p: D columns at 256 + 128 p.
+__host__ __device__ constexpr uint32_t o_col(int p) { return p == 0 ? 256u : 384u; }
 
 template <int T, int D>
 struct Cfg {
@@ -49,7 +66,7 @@ struct Cfg {
   static constexpr int kKTile = T * kQKRowBytes;             // K codes per stage
   static constexpr int kVSub = D * 128;                      // one V sub-tile: D rows x 64 keys
   static constexpr int kVTile = D * T * 2;                   // all V sub-tiles of a stage
-  static constexpr int kStageRaw = kKTile + kVTile + T * 4;
+  static constexpr int kStageRaw = kKTile + kVTile + T * 4;  // + K scales
   static constexpr int kStage = (kStageRaw + 1023) / 1024 * 1024;
   static constexpr int kStages = T == 128 ? 3 : 4;
   static constexpr int kQTile = kRows * kQKRowBytes;
@@ -57,9 +74,11 @@ struct Cfg {
   static constexpr int kOffQ4 = kQTile;
   static constexpr int kOffStage = 2 * kQTile;
   static constexpr int kOffBar = kOffStage + kStages * kStage;
-  // barriers + alignment slack; never below 120 KB so that exactly one CTA (which
-  // owns all 512 TMEM columns) is resident per SM
-  static constexpr int kSmemNeed = kOffBar + 1024 + 1024;
+  static constexpr int kOffX = kOffBar + 1024;               // row-max and epilogue exchanges
+  static constexpr int kXBytes = 2 * 2 * 128 * 4 + 2 * 2 * 2 * 2 * 128 * 4;   // 2 KB + 8 KB
+  // never below 120 KB so that exactly one CTA (which owns all 512 TMEM columns)
+  // is resident per SM
+  static constexpr int kSmemNeed = kOffX + kXBytes + 1024;
   static constexpr int kSmem = kSmemNeed > 120 * 1024 ? kSmemNeed : 120 * 1024;
   static constexpr uint32_t kStageTx = kKTile + kVTile + T * 4;
   static constexpr uint32_t kIdescQK = idesc_i8(kRows, T);
@@ -68,7 +87,7 @@ struct Cfg {
 
 struct Bars {
   uint64_t q_full, q_empty, fin;
-  uint64_t o_done[2];   // P.V of load g completes phase g/2 of o_done[g % 2]
+  uint64_t o_done[kSlots];      // P.V of load g completes phase g/2 of o_done[g % 2]
   uint64_t kv_full[4], kv_empty[4];
   uint64_t s_full[kSlots], s_free[kSlots], p_full[kSlots];
   uint32_t tmem_base;
@@ -131,12 +150,107 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// ---- packed fp32x2 arithmetic (two scores per instruction) ----
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void up2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Softmax pass 1 over N keys of a row: y = float(acc) * s_k as packed pairs, and
+// the maximum over the visible keys (n <= kmax when MASK).
+template <int N, bool MASK>
+__device__ __forceinline__ float scores_and_max(const uint32_t (&r)[N], uint64_t (&y)[N / 2], const float* sk,
+                                                int kmax) {
+  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int q = 0; q < N / 4; ++q) {
+    const float4 s4 = *reinterpret_cast<const float4*>(sk + 4 * q);
+    const uint64_t u01 = pk2(__int2float_rn(static_cast<int>(r[4 * q])), __int2float_rn(static_cast<int>(r[4 * q + 1])));
+    const uint64_t u23 =
+        pk2(__int2float_rn(static_cast<int>(r[4 * q + 2])), __int2float_rn(static_cast<int>(r[4 * q + 3])));
+    y[2 * q] = mul2(u01, pk2(s4.x, s4.y));
+    y[2 * q + 1] = mul2(u23, pk2(s4.z, s4.w));
+    float v0, v1, v2, v3;
+    up2(y[2 * q], v0, v1);
+    up2(y[2 * q + 1], v2, v3);
+    if (MASK) {
+      const int n = 4 * q;
+      v0 = n <= kmax ? v0 : -INFINITY;
+      v1 = n + 1 <= kmax ? v1 : -INFINITY;
+      v2 = n + 2 <= kmax ? v2 : -INFINITY;
+      v3 = n + 3 <= kmax ? v3 : -INFINITY;
+    }
+    mx[(q % 2) * 2] = max3(mx[(q % 2) * 2], v0, v1);
+    mx[(q % 2) * 2 + 1] = max3(mx[(q % 2) * 2 + 1], v2, v3);
+  }
+  return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+}
+
+// Softmax pass 2 over N keys: p = 2^(y * alpha - m) packed to bf16 pairs, their
+// fp32 sum accumulated in `acc`; masked keys (n > kmax when MASK) give 0.
+template <int N, bool MASK>
+__device__ __forceinline__ void probs(const uint64_t (&y)[N / 2], uint64_t al2, uint64_t nm2, int kmax,
+                                      uint32_t (&pk)[N / 2], uint64_t (&acc)[4]) {
+#pragma unroll
+  for (int k = 0; k < N / 2; ++k) {
+    float t0, t1;
+    up2(fma2(y[k], al2, nm2), t0, t1);
+    float e0 = fast_exp2(t0), e1 = fast_exp2(t1);
+    if (MASK) {
+      e0 = 2 * k <= kmax ? e0 : 0.0f;
+      e1 = 2 * k + 1 <= kmax ? e1 : 0.0f;
+    }
+    acc[k % 4] = add2(acc[k % 4], pk2(e0, e1));
+    pk[k] = bf16x2(e0, e1);
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_store_words(uint32_t taddr, const uint32_t (&w)[N]) {
+  static_assert(N == 16 || N == 32, "P stores are 16 or 32 columns");
+  if constexpr (N == 32) {
+    tmem_st32(taddr, w);
+  } else {
+    tmem_st16(taddr, w);
+  }
+}
+
 template <int T, int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ PrefillMaps maps) {
   using C = Cfg<T, D>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base, computed on the __shared__ array itself so that the
+  // compiler keeps every access below in the shared address space
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   Bars* bars = reinterpret_cast<Bars*>(smem + C::kOffBar);
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x / 32;
@@ -146,16 +260,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
     mbar_init(&bars->fin, 1);
-    mbar_init(&bars->o_done[0], 1);
-    mbar_init(&bars->o_done[1], 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
     }
     for (int s = 0; s < kSlots; ++s) {
+      mbar_init(&bars->o_done[s], 1);
       mbar_init(&bars->s_full[s], 1);
       mbar_init(&bars->s_free[s], 1);
-      mbar_init(&bars->p_full[s], 128);
+      mbar_init(&bars->p_full[s], kPairThreads);
     }
     bars->abort = 0;
     fence_mbar_init();
@@ -182,39 +295,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     return reinterpret_cast<float*>(smem + C::kOffStage + s * C::kStage + C::kKTile + C::kVTile);
   };
 
-  if (warp == kProducerWarp) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
+  if (warp >= kSoftmaxWarps) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+    // The producer and MMA loops run on the whole warp, so that their operands are
+    // warp-uniform (uniform registers); one elected lane issues the copies and the
+    // tensor-core ops, and the same lane issues the commits that track them.
+    auto warp_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, a.err));
+    };
+    if (warp == kProducerWarp) {
+      // ---------------------------------------------------------- producer
       uint32_t g = 0, uloc = 0, q_issued = 0;
       bool ok = true;
       for (int w = blockIdx.x; w < a.n_units && ok; w += gridDim.x, ++uloc) {
         const Unit u = unit_of(a, w, C::kQBlocks);
-        if (uloc > 0 && !(ok = mbar_wait(&bars->q_empty, (uloc - 1) & 1, abort, a.err))) break;
+        if (uloc > 0 && !(ok = warp_wait(&bars->q_empty, (uloc - 1) & 1))) break;
         ++q_issued;
         const int qrow = (u.b * a.Hq + u.hq) * a.S + u.i0 * T;
-        mbar_arrive_expect_tx(&bars->q_full, 2 * C::kQTile);
-        tma_load_2d(sQ8, &maps.q8, &bars->q_full, 0, qrow);
-        tma_load_2d(sQ4, &maps.q4, &bars->q_full, 0, qrow);
+        if (elect_one()) {
+          mbar_arrive_expect_tx(&bars->q_full, 2 * C::kQTile);
+          tma_load_2d(sQ8, &maps.q8, &bars->q_full, 0, qrow);
+          tma_load_2d(sQ4, &maps.q4, &bars->q_full, 0, qrow);
+        }
+        __syncwarp();
         LoadSeq seq;
         seq.init(u.i0, u.nq, a.hi[u.hq], a.keep[u.hq]);
         const int64_t grp = static_cast<int64_t>(u.b) * a.Hkv + u.kvh;
         int j, plane;
         while (seq.next(j, plane)) {
           const int st = g % C::kStages;
-          if (g >= static_cast<uint32_t>(C::kStages) &&
-              !(ok = mbar_wait(&bars->kv_empty[st], ((g / C::kStages) - 1) & 1, abort, a.err)))
+          if (g >= static_cast<uint32_t>(C::kStages) && !(ok = warp_wait(&bars->kv_empty[st], ((g / C::kStages) - 1) & 1)))
             break;
-          mbar_arrive_expect_tx(&bars->kv_full[st], C::kStageTx);
           const int krow = static_cast<int>(grp * (plane == 8 ? a.cap8 : static_cast<int64_t>(a.S)) +
                                             static_cast<int64_t>(j) * T);
-          tma_load_2d(sK(st), plane == 8 ? &maps.k8 : &maps.k4, &bars->kv_full[st], 0, krow);
           const int vrow = static_cast<int>((grp * a.nb + j) * D);
-#pragma unroll
-          for (int q = 0; q < T / 64; ++q)
-            tma_load_2d(sV(st) + q * C::kVSub, plane == 8 ? &maps.v8 : &maps.v4, &bars->kv_full[st], 64 * q,
-                        vrow);
           const float* ks = (plane == 8 ? a.k8s : a.k4s) + grp * a.cap + static_cast<int64_t>(j) * T;
-          bulk_load(sScale(st), ks, T * 4, &bars->kv_full[st]);
+          if (elect_one()) {
+            mbar_arrive_expect_tx(&bars->kv_full[st], C::kStageTx);
+            tma_load_2d(sK(st), plane == 8 ? &maps.k8 : &maps.k4, &bars->kv_full[st], 0, krow);
+#pragma unroll
+            for (int q = 0; q < T / 64; ++q)
+              tma_load_2d(sV(st) + q * C::kVSub, plane == 8 ? &maps.v8 : &maps.v4, &bars->kv_full[st], 64 * q,
+                          vrow);
+            bulk_load(sScale(st), ks, T * 4, &bars->kv_full[st]);
+          }
+          __syncwarp();
           ++g;
         }
       }
@@ -222,68 +347,93 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (uint32_t k = (g > static_cast<uint32_t>(C::kStages) ? g - C::kStages : 0); k < g; ++k)
         drain_wait(&bars->kv_full[k % C::kStages], (k / C::kStages) & 1);
       if (q_issued > 0) drain_wait(&bars->q_full, (q_issued - 1) & 1);
-    }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == kMmaWarp) {
+      // ---------------------------------------------------------- MMA issuer
       uint32_t g = 0, uloc = 0;
       bool ok = true;
       const uint32_t q8a = smem_u32(sQ8), q4a = smem_u32(sQ4);
+      // P.V of load gg into the O accumulator of its parity; `first` overwrites.
       auto pv = [&](uint32_t gg, bool first) -> bool {
         const int st = gg % C::kStages, sl = gg % kSlots;
-        if (!mbar_wait(&bars->p_full[sl], (gg / kSlots) & 1, abort, a.err)) return false;
-        tc_fence_after();
         const uint32_t vbase = smem_u32(sV(st));
+        if (!warp_wait(&bars->p_full[sl], (gg / kSlots) & 1)) return false;
+        tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int s = 0; s < T / 16; ++s) {
-          const uint64_t bdesc = sw128_desc(vbase + (s / 4) * C::kVSub + (s % 4) * 32);
-          mma_bf16_ts(tmem + kOCol, tmem + sl * T + s * 8, bdesc, C::kIdescPV, (first && s == 0) ? 0u : 1u);
+          for (int s = 0; s < T / 16; ++s) {
+            const uint64_t bdesc = sw128_desc(vbase + (s / 4) * C::kVSub + (s % 4) * 32);
+            mma_bf16_ts(tmem + o_col(sl), tmem + sl * T + s * 8, bdesc, C::kIdescPV, (first && s == 0) ? 0u : 1u);
+          }
+          mma_commit(&bars->o_done[sl]);
+          mma_commit(&bars->kv_empty[st]);
+          mma_commit(&bars->s_free[sl]);
         }
-        mma_commit(&bars->kv_empty[st]);
-        mma_commit(&bars->s_free[sl]);
-        mma_commit(&bars->o_done[gg % 2]);
+        __syncwarp();
         return true;
       };
       for (int w = blockIdx.x; w < a.n_units && ok; w += gridDim.x, ++uloc) {
         const Unit u = unit_of(a, w, C::kQBlocks);
-        if (!(ok = mbar_wait(&bars->q_full, uloc & 1, abort, a.err))) break;
+        if (!(ok = warp_wait(&bars->q_full, uloc & 1))) break;
         tc_fence_after();
         LoadSeq seq;
         seq.init(u.i0, u.nq, a.hi[u.hq], a.keep[u.hq]);
         int j, plane, l = 0;
+        bool used[kSlots] = {false, false};   // accumulator written in this tile yet?
+        auto pv_next = [&](uint32_t gg) -> bool {
+          const bool first = !used[gg % kSlots];
+          used[gg % kSlots] = true;
+          return pv(gg, first);
+        };
         while (seq.next(j, plane)) {
           const int st = g % C::kStages, sl = g % kSlots;
-          if (!(ok = mbar_wait(&bars->kv_full[st], (g / C::kStages) & 1, abort, a.err))) break;
-          if (g >= static_cast<uint32_t>(kSlots) &&
-              !(ok = mbar_wait(&bars->s_free[sl], ((g / kSlots) - 1) & 1, abort, a.err)))
+          if (!(ok = warp_wait(&bars->kv_full[st], (g / C::kStages) & 1))) break;
+          if (g >= static_cast<uint32_t>(kSlots) && !(ok = warp_wait(&bars->s_free[sl], ((g / kSlots) - 1) & 1)))
             break;
           tc_fence_after();
           const uint32_t abase = plane == 8 ? q8a : q4a;
           const uint32_t bbase = smem_u32(sK(st));
+          if (elect_one()) {
 #pragma unroll
-          for (int k = 0; k < kQKRowBytes / 32; ++k)
-            mma_i8_ss(tmem + sl * T, sw128_desc(abase + 32 * k), sw128_desc(bbase + 32 * k), C::kIdescQK,
-                      k > 0 ? 1u : 0u);
-          mma_commit(&bars->s_full[sl]);
-          if (l > 0 && !(ok = pv(g - 1, l == 1))) break;
+            for (int k = 0; k < kQKRowBytes / 32; ++k)
+              mma_i8_ss(tmem + sl * T, sw128_desc(abase + 32 * k), sw128_desc(bbase + 32 * k), C::kIdescQK,
+                        k > 0 ? 1u : 0u);
+            mma_commit(&bars->s_full[sl]);
+          }
+          __syncwarp();
+          if (l > 0 && !(ok = pv_next(g - 1))) break;
           ++l;
           ++g;
         }
         if (!ok) break;
-        if (l > 0 && !(ok = pv(g - 1, l == 1))) break;
-        mma_commit(&bars->q_empty);
+        if (l > 0 && !(ok = pv_next(g - 1))) break;
+        if (elect_one()) mma_commit(&bars->q_empty);
+        __syncwarp();
       }
       // wait for every tensor-core op this CTA issued before TMEM is released
-      mma_commit(&bars->fin);
+      if (elect_one()) mma_commit(&bars->fin);
+      __syncwarp();
       drain_wait(&bars->fin, 0);
     }
   } else {
-    // ------------------------------------------------------------ softmax (warps 0-3)
-    const int row = threadIdx.x;                        // TMEM lane = query row of the tile
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    uint32_t g = 0;
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    // ------------------------------------------------------------ softmax (warps 0-15)
+    constexpr int TH = T / 2;                 // keys of this thread per load
+    const int pair = warp / 8;                // load parity handled, S slot, O accumulator
+    const int half = (warp / 4) % 2;          // which half of the keys
+    const int sub = warp % 4;                 // TMEM lane quarter
+    const int row = sub * 32 + lane;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(sub * 32) << 16);
+    const uint32_t my_s = lane_addr + pair * T + half * TH;          // S columns of my keys
+    const uint32_t my_p = lane_addr + pair * T + half * (TH / 2);    // P words of my keys
+    const uint32_t my_o = lane_addr + o_col(pair) + half * (D / 2);  // O columns rescaled here
+    const uint32_t pair_bar = 1 + pair * 4 + sub;                    // 64 threads: this row's pair
+    const uint32_t row_bar = 9 + sub;                                // 128 threads: all four of the row
+    // row maxima of loads: [pair][half][row]; epilogue (m, l): [tile parity][pair][half][2][row]
+    float* xmax = reinterpret_cast<float*>(smem + C::kOffX);
+    float* xepi = xmax + 2 * 2 * 128;
+    uint32_t g = 0, uloc = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < a.n_units && ok; w += gridDim.x) {
+    for (int w = blockIdx.x; w < a.n_units && ok; w += gridDim.x, ++uloc) {
       const Unit u = unit_of(a, w, C::kQBlocks);
       const int qb = row / T;
       const int rl = row % T;
@@ -293,114 +443,137 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float a8 = valid ? a.q8s[qrow] * a.qk_log2 : 0.0f;
       const float a4 = valid ? a.q4s[qrow] * a.qk_log2 : 0.0f;
       const int hi = a.hi[u.hq], keep = a.keep[u.hq];
-      float m_run = -INFINITY, l_run = 0.0f;
+      float m_run = -INFINITY, l_run = 0.0f;     // m_run: shared by both halves of the pair
+      int64_t g_mine = -1;                        // last load of this tile handled by this pair
       LoadSeq seq;
       seq.init(u.i0, u.nq, hi, keep);
       int j, plane;
       while (seq.next(j, plane)) {
-        const int st = g % C::kStages, sl = g % kSlots;
+        if (static_cast<int>(g % kSlots) != pair) { ++g; continue; }
+        const int st = g % C::kStages;
         if (!(ok = mbar_wait(&bars->kv_full[st], (g / C::kStages) & 1, abort, a.err))) break;
-        if (!(ok = mbar_wait(&bars->s_full[sl], (g / kSlots) & 1, abort, a.err))) break;
+        if (!(ok = mbar_wait(&bars->s_full[pair], (g / kSlots) & 1, abort, a.err))) break;
+        // QK of this load waited for the P.V two loads back, which used this slot and
+        // this accumulator: the accumulator is final for now and may be rescaled.
         tc_fence_after();
-        const int act = valid ? tile_action(ir, j, hi, keep) : ACT_NONE;
-        const uint32_t s_addr = lane_addr + sl * T;
+        g_mine = g;
+        const int act = valid ? tile_action(ir, j, hi, keep) : ACT_NONE;   // uniform over the warp pair
         if (act == plane) {
-          uint32_t r[T];
+          const int kmax = (j == ir) ? rl - half * TH : TH;   // my keys [0, kmax] are visible
+          uint32_t r[TH];
 #pragma unroll
-          for (int c = 0; c < T / 32; ++c) tmem_ld32(s_addr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
-          tmem_wait_ld();
-          const float* ks = sScale(st);
+          for (int c = 0; c < TH / 32; ++c) tmem_ld32(my_s + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+          const float* sk = sScale(st) + half * TH;
           const float alpha = plane == 8 ? a8 : a4;
-          const bool diag = (j == ir);
-          float mx = -INFINITY;
-#pragma unroll
-          for (int n = 0; n < T; ++n) {
-            float y = __int2float_rn(static_cast<int>(r[n])) * ks[n];
-            if (diag && n > rl) y = -INFINITY;
-            mx = fmaxf(mx, y);
-            r[n] = __float_as_uint(y);
-          }
-          const float m_tile = mx * alpha;
+          tmem_wait_ld();
+          uint64_t y[TH / 2];
+          const bool masked = kmax < TH - 1;
+          const float m_half = masked ? scores_and_max<TH, true>(r, y, sk, kmax) : scores_and_max<TH, false>(r, y, sk, kmax);
+          // both halves have read their S (tcgen05.wait::ld above) before either stores P
+          float* xb = xmax + pair * 256;
+          xb[half * 128 + row] = m_half;
+          named_bar_sync(pair_bar, 64);
+          const float m_tile = fmaxf(m_half, xb[(1 - half) * 128 + row]) * alpha;
           const bool raise = m_tile > m_run + kRescaleLog2;
           const float sc = raise ? fast_exp2(m_run - m_tile) : 1.0f;
-          // TMEM loads/stores are warp-collective: the whole warp rescales its O rows
-          // when any lane must (lanes that need not use the factor 1).
-          if (__any_sync(0xffffffffu, raise && l_run > 0.0f)) {
-            // O holds earlier loads of this tile: wait for the previous P.V first.
-            if (!(ok = mbar_wait(&bars->o_done[(g - 1) % 2], ((g - 1) / 2) & 1, abort, a.err))) break;
-            tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t o[32];
-              tmem_ld32(lane_addr + kOCol + 32 * c, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * sc);
-              tmem_st32(lane_addr + kOCol + 32 * c, o);
-            }
-          }
+          const bool rescale_o = raise && m_run != -INFINITY;
           if (raise) {
             l_run *= sc;
             m_run = m_tile;
           }
-          float sum = 0.0f;
-#pragma unroll
-          for (int c = 0; c < T / 64; ++c) {
-            uint32_t pk[32];
-#pragma unroll
-            for (int k = 0; k < 32; ++k) {
-              const int n = 64 * c + 2 * k;
-              const float y0 = __uint_as_float(r[n]), y1 = __uint_as_float(r[n + 1]);
-              const float p0 = (diag && n > rl) ? 0.0f : fast_exp2(fmaf(y0, alpha, -m_run));
-              const float p1 = (diag && n + 1 > rl) ? 0.0f : fast_exp2(fmaf(y1, alpha, -m_run));
-              sum += p0 + p1;
-              const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-              pk[k] = *reinterpret_cast<const uint32_t*>(&h);
-            }
-            tmem_st32(s_addr + 32 * c, pk);
+          const uint64_t al2 = pk2(alpha, alpha), nm2 = pk2(-m_run, -m_run);
+          uint64_t acc[4] = {0, 0, 0, 0};
+          {
+            uint32_t pk[TH / 2];
+            if (masked) probs<TH, true>(y, al2, nm2, kmax, pk, acc);
+            else probs<TH, false>(y, al2, nm2, kmax, pk, acc);
+            tmem_store_words<TH / 2>(my_p, pk);
           }
-          l_run += sum;
+          float s0, s1;
+          up2(add2(add2(acc[0], acc[1]), add2(acc[2], acc[3])), s0, s1);
+          l_run += s0 + s1;
+          // Rescale this half's O columns when the maximum rose (before P.V of this load
+          // may start). TMEM loads/stores are warp-collective: the whole warp takes part
+          // when any lane must, lanes that need not using the factor 1.
+          if (__any_sync(0xffffffffu, rescale_o)) {
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) {
+              uint32_t o[32];
+              tmem_ld32(my_o + 32 * c, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * sc);
+              tmem_st32(my_o + 32 * c, o);
+            }
+          }
         } else {
-          uint32_t z[32];
+          uint32_t z[TH / 2];
 #pragma unroll
-          for (int k = 0; k < 32; ++k) z[k] = 0u;
-#pragma unroll
-          for (int c = 0; c < T / 64; ++c) tmem_st32(s_addr + 32 * c, z);
+          for (int k = 0; k < TH / 2; ++k) z[k] = 0u;
+          tmem_store_words<TH / 2>(my_p, z);
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars->p_full[sl]);
+        mbar_arrive(&bars->p_full[pair]);
         ++g;
       }
       if (!ok) break;
-      // epilogue: wait for the last P.V of the tile, normalise, store. Having seen QK of
-      // load gl complete, every P.V up to gl-2 is complete, so o_done[gl % 2] is at most
-      // one phase short of the one awaited and its parity is unambiguous.
-      const uint32_t gl = g - 1;
-      if (!(ok = mbar_wait(&bars->o_done[gl % 2], (gl / 2) & 1, abort, a.err))) break;
-      tc_fence_after();
-      const float inv_l = valid ? 1.0f / l_run : 0.0f;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(lane_addr + kOCol + 32 * c, o);
-        tmem_wait_ld();
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(a.O + qrow * D + 32 * c);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            uint32_t wv[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(o[8 * k + 2 * e]) * inv_l,
-                                                             __uint_as_float(o[8 * k + 2 * e + 1]) * inv_l);
-              wv[e] = *reinterpret_cast<const uint32_t*>(&h);
-            }
-            dst[k] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-          }
-        }
+      // Epilogue. The last P.V into this pair's accumulator: its QK was seen, so the
+      // P.V two loads earlier is complete and o_done[pair] is at most one phase short.
+      if (g_mine >= 0) {
+        const uint32_t gm = static_cast<uint32_t>(g_mine);
+        if (!(ok = mbar_wait(&bars->o_done[pair], (gm / kSlots) & 1, abort, a.err))) break;
+        tc_fence_after();
       }
-      if (valid) a.LSE[qrow] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+      float* xe = xepi + (uloc & 1) * (2 * 2 * 2 * 128);
+      auto slot = [&](int p, int h, int v) { return xe + ((p * 2 + h) * 2 + v) * 128 + row; };
+      *slot(pair, half, 0) = m_run;
+      *slot(pair, half, 1) = l_run;
+      named_bar_sync(row_bar, 128);
+      const float m0 = *slot(0, 0, 0), m1 = *slot(1, 0, 0);
+      const float l0 = *slot(0, 0, 1) + *slot(0, 1, 1);
+      const float l1 = *slot(1, 0, 1) + *slot(1, 1, 1);
+      const float m_all = fmaxf(m0, m1);
+      // an accumulator that saw no kept key in this tile (l = 0) may hold stale values
+      const bool use0 = l0 > 0.0f, use1 = l1 > 0.0f;
+      const float w0 = use0 ? fast_exp2(m0 - m_all) : 0.0f;
+      const float w1 = use1 ? fast_exp2(m1 - m_all) : 0.0f;
+      const float l_tot = l0 * w0 + l1 * w1;
+      const float inv_l = valid ? 1.0f / l_tot : 0.0f;
+      const float f0 = w0 * inv_l, f1 = w1 * inv_l;
+      // this thread writes output columns [quarter * D/4, (quarter+1) * D/4)
+      const int quarter = pair * 2 + half;
+      constexpr int QC = D / 4;
+      uint32_t o0[32], o1[32];
+      if constexpr (QC == 32) {
+        tmem_ld32(lane_addr + o_col(0) + quarter * QC, o0);
+        tmem_ld32(lane_addr + o_col(1) + quarter * QC, o1);
+      } else {
+        tmem_ld16(lane_addr + o_col(0) + quarter * QC, o0);
+        tmem_ld16(lane_addr + o_col(1) + quarter * QC, o1);
+      }
+      tmem_wait_ld();
+      if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(a.O + qrow * D + quarter * QC);
+#pragma unroll
+        for (int k = 0; k < QC / 8; ++k) {
+          uint32_t wv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i0 = 8 * k + 2 * e;
+            const float v0 = (use0 ? __uint_as_float(o0[i0]) * f0 : 0.0f) + (use1 ? __uint_as_float(o1[i0]) * f1 : 0.0f);
+            const float v1 =
+                (use0 ? __uint_as_float(o0[i0 + 1]) * f0 : 0.0f) + (use1 ? __uint_as_float(o1[i0 + 1]) * f1 : 0.0f);
+            wv[e] = bf16x2(v0, v1);
+          }
+          dst[k] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+        if (quarter == 0) a.LSE[qrow] = (m_all + log2f(l_tot)) * 0.69314718055994531f;
+      }
+      // All four threads of the row read both accumulators: none may let the next
+      // tile's first P.V (which overwrites them) start before the others have read.
+      tc_fence_before();
+      named_bar_sync(row_bar, 128);
     }
   }
 
