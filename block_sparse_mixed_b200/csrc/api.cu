@@ -162,9 +162,9 @@ DecodeLayout decode_layout(int B, int Hq, int Hkv, int D) {
   const size_t items = groups * kMaxSplitsPerGroup;
   size_t off = 0;
   L.ctrl = off; off += align_up(64);
-  L.counts = off; off += align_up(groups * 4);
+  L.counts = off; off += align_up(groups * kDecodeSlices * 4);
   L.part_o = off; off += align_up(items * G * D * 4);
-  L.part_ml = off; off += align_up(items * G * 2 * 4);
+  L.part_ml = off; off += align_up(items * kDecodeSlices * G * 4);
   L.total = off;
   return L;
 }
@@ -403,8 +403,9 @@ int tria_decode(const void* q, const tria_kv_cache* cache, const int32_t* kv_len
   a.k8 = cache->k8; a.k4 = cache->k4; a.k8s = cache->k8_scale; a.k4s = cache->k4_scale;
   a.v8 = cache->v8; a.v4 = cache->v4; a.v8s = cache->v8_scale; a.v4s = cache->v4_scale;
   a.part_o = reinterpret_cast<float*>(ws + L.part_o);
-  a.part_ml = reinterpret_cast<float*>(ws + L.part_ml);
+  a.part_lse = reinterpret_cast<float*>(ws + L.part_ml);
   a.group_count = reinterpret_cast<int*>(ws + L.counts);
+  a.work = reinterpret_cast<int*>(ws + L.ctrl) + 4;
   a.O = static_cast<__nv_bfloat16*>(O); a.LSE = LSE;
   a.err = reinterpret_cast<int*>(ws + L.ctrl);
   a.n_groups = groups;
@@ -420,13 +421,15 @@ int tria_decode(const void* q, const tria_kv_cache* cache, const int32_t* kv_len
 
   DecodeMaps maps;
   const uint64_t rows = static_cast<uint64_t>(groups) * cache->capacity;
+  if (rows > static_cast<uint64_t>(INT32_MAX)) return TRIA_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
   const bool ok = make_map(&maps.k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, cache->k8, D, rows, D, T) &&
                   make_map(&maps.k4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, cache->k4, D / 2, rows, D / 2, T) &&
                   make_map(&maps.v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, cache->v8, D, rows, D, T) &&
                   make_map(&maps.v4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, cache->v4, D / 2, rows, D / 2, T);
   if (!ok) return TRIA_ERR_CUDA;
-  if (cudaMemsetAsync(ws, 0, L.counts + groups * 4, st) != cudaSuccess) return TRIA_ERR_CUDA;
-  return cuda_status(launch_decode(a, maps, st));
+  if (cudaMemsetAsync(ws, 0, L.counts + static_cast<size_t>(groups) * kDecodeSlices * 4, st) != cudaSuccess)
+    return TRIA_ERR_CUDA;
+  return cuda_status(launch_decode(a, maps, dev.sms, st));
 }
 
 int tria_workspace_status(const void* workspace, void* stream) {

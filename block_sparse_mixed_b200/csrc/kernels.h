@@ -12,6 +12,7 @@ constexpr int kMaxHeads = 256;     // Hq limit (policy arrays travel in kernel p
 constexpr int kMaxBatch = 1024;    // decode: kv_len travels in kernel parameters
 constexpr int kMaxGroups = 2048;   // decode: B * Hkv
 constexpr int kQKRowBytes = 128;   // Q/K code rows as the tensor cores read them (D padded to 128)
+constexpr int kDecodeSlices = 8;   // decode: most compute warps per CTA (each owns a slice of the output)
 
 // Codec over rows. Output row of input row r:
 //   (r / rows_per_group) * group_stride + start + r % rows_per_group.
@@ -80,9 +81,10 @@ struct DecodeArgs {
   const __nv_bfloat16* q; // [B, Hq, D]
   const int8_t* k8; const uint8_t* k4; const float* k8s; const float* k4s;
   const int8_t* v8; const uint8_t* v4; const float* v8s; const float* v4s;
-  float* part_o;          // [items, G, D]
-  float* part_ml;         // [items, G, 2]
-  int* group_count;       // [groups] items finished; zero before the launch
+  float* part_o;          // [items, G, D] normalised partial outputs
+  float* part_lse;        // [items, kDecodeSlices, G] partial log2-sum-exp, one copy per slice
+  int* group_count;       // [groups, kDecodeSlices] items whose slice is written; zero before the launch
+  int* work;              // next work item (dynamic scheduling); zero before the launch
   __nv_bfloat16* O;
   float* LSE;
   int* err;
@@ -97,6 +99,6 @@ cudaError_t launch_quant_rows(const QuantArgs& a, int D, cudaStream_t stream);
 cudaError_t launch_prepare(const PrepareArgs& a, int D, int T, int groups, int nblocks, cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillArgs& a, const PrefillMaps& maps, int D, int T, int num_sms,
                            cudaStream_t stream);
-cudaError_t launch_decode(const DecodeArgs& a, const DecodeMaps& maps, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs& a, const DecodeMaps& maps, int num_sms, cudaStream_t stream);
 
 }  // namespace tria

@@ -166,15 +166,44 @@ DECODE_CASES = {
     "t64_d64": (2, 4, 1, 64, 64, 640, [640, 65], [(1, 3), (2, 9), (0, 1), (3, 4)]),
     "single_block": (2, 2, 2, 128, 128, 256, [1, 128], [(1, 4), (0, 2)]),
     "g16": (1, 16, 1, 128, 64, 1024, [777], [(h % 4, 2 + h) for h in range(16)]),
+    "g12_t128": (1, 12, 1, 128, 128, 2048, [1999], [(h % 5, 1 + 2 * h) for h in range(12)]),
+    "t128_d64_g8": (2, 16, 2, 64, 128, 1536, [1536, 700], [((3 * h) % 4, 2 + (h % 7)) for h in range(16)]),
 }
+
+
+def test_decode_large_values(T, oracle_mod):
+    """V of magnitude ~500: 4-bit V scales near 200 force the running maximum to
+    move more often so that P * s_v stays finite in fp16."""
+    B, Hq, Hkv, D, Tb, cap = 2, 8, 2, 128, 128, 4096
+    hi = np.array([1, 2, 0, 3, 1, 4, 2, 0], np.int32)
+    keep = np.array([6, 9, 3, 32, 2, 12, 20, 5], np.int32)
+    q, K = seeded((B, Hq, D), 71), seeded((B, Hkv, cap, D), 72)
+    V = (seeded((B, Hkv, cap, D), 73).float() * 128.0).to(torch.bfloat16)
+    kv = np.array([4096, 3001], np.int32)
+    O, L = run_decode(T, q, K, V, Tb, kv, hi, keep)
+    O_ref, L_ref = oracle_mod.decode(q, K, V, Tb, kv, hi, keep)
+    # outputs scale with V: the bound is relative to the V magnitude (bf16 rounding of O included)
+    ref = torch.from_numpy(O_ref).double()
+    err = (O.double().cpu() - ref).abs()
+    assert float(err.max()) <= 128.0 * 1e-2 + 2.0 ** -8 * float(ref.abs().max()), float(err.max())
+    compare_lse(L, L_ref, "large_values")
 
 
 def run_decode(T, q, K, V, Tb, kv_len, hi, keep):
     B, Hkv, cap, D = K.shape
     cache = T.CompressedKVCache(B, Hkv, D, Tb, cap)
     T.tria_quantize_kv(K.cuda(), V.cuda(), cache)
-    O, L = T.tria_decode(q.cuda(), cache, kv_len, hi, keep)
-    torch.cuda.synchronize()
+    qd = q.cuda()
+    ws = torch.empty(T.tria_decode_workspace_bytes(B, q.shape[1], Hkv, D, Tb, cap), dtype=torch.uint8, device="cuda")
+    for _ in range(2):   # a second call on the same workspace must work as well
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        O, L = T.tria_decode(qd, cache, kv_len, hi, keep, workspace=ws)
+        t1.record()
+        torch.cuda.synchronize()
+        assert T.tria_workspace_status(ws) == 0
+        # a pipeline wait that ran out would take seconds even if it left no error
+        assert t0.elapsed_time(t1) < 500.0, t0.elapsed_time(t1)
     return O, L
 
 
