@@ -170,7 +170,7 @@ def run_gpu(args, rank, world, device):
         Ld = torch.empty((w.B, w.Hq), dtype=torch.float32, device=device)
         work = prefill_work(w, hi, keep, tria)
         dbytes = decode_bytes(w.B, w.Hq, w.Hkv, w.D, w.T, kv_len, hi, keep)
-        launches_per_step = 2 + 3 + 1
+        launches_per_step = 2 + 3 + 2
 
         def step(times):
             e = [ev() for _ in range(4)]
@@ -192,7 +192,7 @@ def run_gpu(args, rank, world, device):
         Od = torch.empty_like(q)
         Ld = torch.empty((w.B, w.Hq), dtype=torch.float32, device=device)
         dbytes = decode_bytes(w.B, w.Hq, w.Hkv, w.D, w.T, kv_len, hi, keep)
-        launches_per_step = 1
+        launches_per_step = 2
 
         def step(times):
             e = [ev() for _ in range(2)]

@@ -19,7 +19,6 @@ namespace tria {
 namespace {
 
 constexpr size_t kAlign = 256;
-constexpr int kMaxSplitsPerGroup = 32;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -152,19 +151,24 @@ int check_dims(const tria_dims* d) {
 }
 
 struct DecodeLayout {
-  size_t ctrl, counts, part_o, part_ml, total;
+  size_t ctrl, part_o, part_ml, total;
+  int max_items;
 };
+
+// Decode work items are bounded so that the partials fit a workspace sized from
+// the shapes alone: at least two per group, at least 512 in all.
+int decode_max_items(int groups) { return std::max(2 * groups, 512); }
 
 DecodeLayout decode_layout(int B, int Hq, int Hkv, int D) {
   DecodeLayout L{};
   const size_t groups = static_cast<size_t>(B) * Hkv;
   const size_t G = static_cast<size_t>(Hq / Hkv);
-  const size_t items = groups * kMaxSplitsPerGroup;
+  L.max_items = decode_max_items(static_cast<int>(groups));
+  const size_t parts = static_cast<size_t>(L.max_items) * kDecodeSlices;
   size_t off = 0;
   L.ctrl = off; off += align_up(64);
-  L.counts = off; off += align_up(groups * kDecodeSlices * 4);
-  L.part_o = off; off += align_up(items * G * D * 4);
-  L.part_ml = off; off += align_up(items * kDecodeSlices * G * 4);
+  L.part_o = off; off += align_up(parts * G * D * 4);
+  L.part_ml = off; off += align_up(parts * G * 2 * 4);
   L.total = off;
   return L;
 }
@@ -390,9 +394,18 @@ int tria_decode(const void* q, const tria_kv_cache* cache, const int32_t* kv_len
       nkept[b * Hkv + k] = ib == 0 ? 1 : 1 + (ib - jb + 1);
       total += nkept[b * Hkv + k];
     }
-  const int64_t target_items = static_cast<int64_t>(dev.sms) * 2 * 6;
-  int bps = static_cast<int>(std::max<int64_t>(4, (total + target_items - 1) / target_items));
-  for (int g = 0; g < groups; ++g) bps = std::max(bps, (nkept[g] + kMaxSplitsPerGroup - 1) / kMaxSplitsPerGroup);
+  // about six items per SM; items of one group are consecutive runs of its kept blocks
+  const int64_t target_items = static_cast<int64_t>(dev.sms) * 6;
+  int bps = static_cast<int>(std::max<int64_t>(1, (total + target_items - 1) / target_items));
+  auto count_items = [&](int b) {
+    int64_t n = 0;
+    for (int g = 0; g < groups; ++g) n += (nkept[g] + b - 1) / b;
+    return n;
+  };
+  // sum over groups of ceil(n_g / bps) <= total / bps + groups
+  if (L.max_items > groups)
+    bps = std::max<int64_t>(bps, (total + (L.max_items - groups) - 1) / (L.max_items - groups));
+  while (count_items(bps) > L.max_items) ++bps;
 
   DecodeArgs a{};
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.G = G; a.D = D; a.T = T;
@@ -403,8 +416,7 @@ int tria_decode(const void* q, const tria_kv_cache* cache, const int32_t* kv_len
   a.k8 = cache->k8; a.k4 = cache->k4; a.k8s = cache->k8_scale; a.k4s = cache->k4_scale;
   a.v8 = cache->v8; a.v4 = cache->v4; a.v8s = cache->v8_scale; a.v4s = cache->v4_scale;
   a.part_o = reinterpret_cast<float*>(ws + L.part_o);
-  a.part_lse = reinterpret_cast<float*>(ws + L.part_ml);
-  a.group_count = reinterpret_cast<int*>(ws + L.counts);
+  a.part_ml = reinterpret_cast<float*>(ws + L.part_ml);
   a.work = reinterpret_cast<int*>(ws + L.ctrl) + 4;
   a.O = static_cast<__nv_bfloat16*>(O); a.LSE = LSE;
   a.err = reinterpret_cast<int*>(ws + L.ctrl);
@@ -427,8 +439,7 @@ int tria_decode(const void* q, const tria_kv_cache* cache, const int32_t* kv_len
                   make_map(&maps.v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, cache->v8, D, rows, D, T) &&
                   make_map(&maps.v4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, cache->v4, D / 2, rows, D / 2, T);
   if (!ok) return TRIA_ERR_CUDA;
-  if (cudaMemsetAsync(ws, 0, L.counts + static_cast<size_t>(groups) * kDecodeSlices * 4, st) != cudaSuccess)
-    return TRIA_ERR_CUDA;
+  if (cudaMemsetAsync(ws + L.ctrl, 0, 64, st) != cudaSuccess) return TRIA_ERR_CUDA;   // error word, work counter
   return cuda_status(launch_decode(a, maps, dev.sms, st));
 }
 

@@ -12,7 +12,7 @@ constexpr int kMaxHeads = 256;     // Hq limit (policy arrays travel in kernel p
 constexpr int kMaxBatch = 1024;    // decode: kv_len travels in kernel parameters
 constexpr int kMaxGroups = 2048;   // decode: B * Hkv
 constexpr int kQKRowBytes = 128;   // Q/K code rows as the tensor cores read them (D padded to 128)
-constexpr int kDecodeSlices = 8;   // decode: most compute warps per CTA (each owns a slice of the output)
+constexpr int kDecodeSlices = 8;   // decode: most compute warps per CTA (each writes its own partial)
 
 // Codec over rows. Output row of input row r:
 //   (r / rows_per_group) * group_stride + start + r % rows_per_group.
@@ -81,9 +81,10 @@ struct DecodeArgs {
   const __nv_bfloat16* q; // [B, Hq, D]
   const int8_t* k8; const uint8_t* k4; const float* k8s; const float* k4s;
   const int8_t* v8; const uint8_t* v4; const float* v8s; const float* v4s;
-  float* part_o;          // [items, G, D] normalised partial outputs
-  float* part_lse;        // [items, kDecodeSlices, G] partial log2-sum-exp, one copy per slice
-  int* group_count;       // [groups, kDecodeSlices] items whose slice is written; zero before the launch
+  int slices;             // compute warps per CTA: partials per item
+  int stages;             // ring stages (from the shared memory available)
+  float* part_o;          // [items, slices, G, D] unnormalised partial outputs (x 64)
+  float* part_ml;         // [items, slices, G, 2] partial (max in log2 units, sum)
   int* work;              // next work item (dynamic scheduling); zero before the launch
   __nv_bfloat16* O;
   float* LSE;
