@@ -81,6 +81,8 @@ struct DecodeArgs {
   const __nv_bfloat16* q; // [B, Hq, D]
   const int8_t* k8; const uint8_t* k4; const float* k8s; const float* k4s;
   const int8_t* v8; const uint8_t* v4; const float* v8s; const float* v4s;
+  uint32_t magic[8];      // bit masks and biases of the code conversions, filled by the launcher
+                          // (as kernel parameters they stay register operands of one lop3 each)
   int slices;             // compute warps per CTA: partials per item
   int stages;             // ring stages (from the shared memory available)
   float* part_o;          // [items, slices, G, D] unnormalised partial outputs (x 64)
