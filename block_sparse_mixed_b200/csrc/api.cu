@@ -396,7 +396,8 @@ int tria_decode(const void* q, const tria_kv_cache* cache, const int32_t* kv_len
     }
   // about six items per SM; items of one group are consecutive runs of its kept blocks
   const int64_t target_items = static_cast<int64_t>(dev.sms) * 6;
-  int bps = static_cast<int>(std::max<int64_t>(1, (total + target_items - 1) / target_items));
+  // (at least 4 blocks: small problems are bound by latency, and fewer partials merge faster)
+  int bps = static_cast<int>(std::max<int64_t>(4, (total + target_items - 1) / target_items));
   auto count_items = [&](int b) {
     int64_t n = 0;
     for (int g = 0; g < groups; ++g) n += (nkept[g] + b - 1) / b;
