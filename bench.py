@@ -57,33 +57,74 @@ def load_peaks():
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+    """SM clock and clock-event (throttle) reasons sampled during the timed region.
 
+    NVML (read-only queries) every 5 ms from a thread; nvidia-smi every 200 ms when
+    NVML is not importable."""
+
+    # NVML clock-event reason bits
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int):
         self.idx = device_index
-        self.samples = []
+        self.sm, self.mx, self.reasons = [], [], set()
+        self._nv = None
         self._stop = threading.Event()
         self._t = None
 
-    def _run(self):
+    def _run_nvml(self, nv):
+        h = nv.nvmlDeviceGetHandleByIndex(self.idx)
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self._stop.is_set():
+            self.sm.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+            self.mx.append(float(mx))
+            bits = int(get_reasons(h))
+            self.reasons.update(name for bit, name in self.REASONS.items() if bits & bit)
+            self._stop.wait(0.005)
+
+    def _run_smi(self):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         while not self._stop.is_set():
             try:
                 out = subprocess.run(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
                                       "--format=csv,noheader,nounits"], capture_output=True, text=True,
                                      timeout=5).stdout.strip()
-                if out:
-                    self.samples.append([f.strip() for f in out.split(",")])
+                f = [x.strip() for x in out.split(",")]
+                if len(f) >= 9:
+                    self.sm.append(float(f[1]))
+                    self.mx.append(float(f[2]))
+                    self.reasons.update(names[k] for k in range(4) if f[5 + k].lower() == "active")
             except Exception:
                 pass
             self._stop.wait(0.2)
 
+    def _run(self):
+        if self._nv is None:
+            self._run_smi()
+            return
+        try:
+            self._run_nvml(self._nv)
+        finally:
+            self._nv.nvmlShutdown()
+
     def __enter__(self):
+        try:   # NVML is brought up before the timed region starts
+            import pynvml as nv
+            nv.nvmlInit()
+            self._nv = nv
+        except Exception:
+            self._nv = None
         self._t = threading.Thread(target=self._run, daemon=True)
         self._t.start()
+        t0 = time.time()
+        while not self.sm and time.time() - t0 < 2.0:   # first sample taken before timing starts
+            time.sleep(0.001)
         return self
 
     def __exit__(self, *exc):
@@ -91,15 +132,33 @@ class ClockSampler:
         self._t.join(timeout=10)
 
     def summary(self):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
-        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[k] for s in self.samples for k in range(4)
-                          if len(s) > 5 + k and s[5 + k].strip().lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(self.samples)}
+        if not self.sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(self.sm), "sm_max_mhz": max(self.mx),
+                "reasons": sorted(self.reasons), "samples": len(self.sm)}
+
+
+# ---------------------------------------------------------------- ncu traffic
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch (read + write) of `kernel` on `workload`, from the ncu
+    summary table in profiles/traffic.md, or None when there is no entry or the
+    kernel source has changed since the counters were taken (hash mismatch)."""
+    import hashlib
+    import re
+    table = ROOT / "profiles" / "traffic.md"
+    if not table.exists():
+        return None
+    for line in table.read_text().splitlines():
+        m = re.match(r"^\|\s*(\w+)\s*\|\s*([\w.]+)\s*\|\s*([0-9.eE+]+)\s*\|\s*([\w/.]+)\s*\|\s*([0-9a-f]{12})\s*\|",
+                     line)
+        if not m or m.group(1) != kernel or m.group(2) != workload:
+            continue
+        src = ROOT / "block_sparse_mixed_b200" / "csrc" / m.group(4)
+        if not src.exists() or hashlib.sha256(src.read_bytes()).hexdigest()[:12] != m.group(5):
+            return None
+        return float(m.group(3))
+    return None
 
 
 # ---------------------------------------------------------------- accounting
@@ -173,14 +232,17 @@ def run_gpu(args, rank, world, device):
         launches_per_step = 2 + 3 + 2
 
         def step(times):
-            e = [ev() for _ in range(4)]
+            # tria_prefill in its two halves, so that the fused kernel is timed alone
+            e = [ev() for _ in range(5)]
             e[0].record(stream)
             tria.tria_quantize_kv(K, V, cache)
             e[1].record(stream)
-            tria.tria_prefill(Q, cache, hi, keep, workspace=ws, O=O, LSE=LSE)
+            tria.tria_prefill_prepare(Q, cache, ws)
             e[2].record(stream)
-            tria.tria_decode(q_last, cache, kv_len, hi, keep, workspace=dws, O=Od, LSE=Ld)
+            tria.tria_prefill_attend(cache, hi, keep, ws, O, LSE)
             e[3].record(stream)
+            tria.tria_decode(q_last, cache, kv_len, hi, keep, workspace=dws, O=Od, LSE=Ld)
+            e[4].record(stream)
             times.append(e)
     else:
         q, K, V, kv_len = W.decode_inputs(w, device=device)
@@ -235,22 +297,25 @@ def run_gpu(args, rank, world, device):
     if w.kind == "prefill":
         tokens = w.B * w.S
         res["value"] = tokens * world / (step_ms_max / 1e3)
-        q_ms, p_ms, d_ms = (float(seg[:, i].mean()) for i in range(3))
+        q_ms, prep_ms, att_ms, d_ms = (float(seg[:, i].mean()) for i in range(4))
+        p_ms = prep_ms + att_ms
         p_i8 = peaks["bf16_tflops"] * INT8_OVER_BF16
         t_roof = work["ops_int8"] / (p_i8 * 1e12) + work["flop_bf16"] / (peaks["bf16_tflops"] * 1e12)
         ops = work["ops_int8"] + work["flop_bf16"]
-        achieved = ops / (p_ms / 1e3) / 1e12
+        achieved = ops / (att_ms / 1e3) / 1e12
         peak = ops / t_roof / 1e12
-        res["roofline"] = {"bound": "tensor", "kernel": "tria_prefill (Q codec + operand prep + fused tcgen05)",
+        res["roofline"] = {"bound": "tensor", "kernel": "prefill_kernel (tria_prefill_attend, fused tcgen05)",
                            "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                           "traffic": None,
+                           "traffic": recorded_traffic("prefill_kernel", w.name),
                            "peak_note": f"int8 {p_i8:.1f} TOPS (= {peak_src} bf16 burst x {INT8_OVER_BF16:g} nominal "
                                         f"ratio) for QK, bf16 {peaks['bf16_tflops']} TFLOP/s ({peak_src}) for P.V"}
         qkv_bytes = 2 * (K.numel() * 2) + 2 * (K.numel() + K.numel() // 2) + 4 * 4 * K.numel() // w.D
         res["rows"] = {
             "quantize_kv": {"ms": q_ms, "GB/s": qkv_bytes / (q_ms / 1e3) / 1e9,
                             "frac_hbm": qkv_bytes / (q_ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
-            "prefill": {"ms": p_ms, "TOPS_kept": achieved, "frac_roofline": achieved / peak, **work},
+            "prefill": {"ms": p_ms, "prepare_ms": prep_ms, "attend_ms": att_ms, "TOPS_kept": achieved,
+                        "frac_roofline": achieved / peak,
+                        "TOPS_kept_whole_call": ops / (p_ms / 1e3) / 1e12, **work},
             "decode": {"ms": d_ms, "kept_bytes": dbytes, "GB/s": dbytes / (d_ms / 1e3) / 1e9,
                        "frac_hbm": dbytes / (d_ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
         }
@@ -258,8 +323,10 @@ def run_gpu(args, rank, world, device):
         d_ms = float(seg[:, 0].mean())
         gbs = dbytes / (d_ms / 1e3) / 1e9
         res["value"] = gbs * world
-        res["roofline"] = {"bound": "hbm", "kernel": "tria_decode", "achieved": gbs, "peak": peaks["hbm_gbs"],
-                           "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+        res["roofline"] = {"bound": "hbm", "kernel": "tria_decode (decode_kernel + decode_merge_kernel)",
+                           "achieved": gbs, "peak": peaks["hbm_gbs"],
+                           "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                           "traffic": recorded_traffic("decode_kernel", w.name),
                            "peak_note": f"HBM copy bandwidth ({peak_src})"}
         res["rows"] = {"decode": {"ms": d_ms, "kept_bytes": dbytes}}
     res["gpu_launches"] = launches_per_step * args.steps
@@ -342,7 +409,8 @@ def oracle_sample(w: W.Workload, budget_s: float, seed: int = 0):
             n_rows = int(min(8192, max(64, n_rows * 2 if el < budget_s / 4 else n_rows)))
         elapsed = time.perf_counter() - t0
         rows_per_s = done / elapsed
-        return rows_per_s / w.Hq, "tokens/s", f"{done} random query rows (of {w.B * w.Hq * w.S}), " \
+        return rows_per_s / w.Hq, "tokens/s", f"{done} query rows drawn at random with replacement " \
+                                               f"(the workload has {w.B * w.Hq * w.S}), " \
                                                f"{elapsed:.1f} s; tokens/s = rows/s / Hq", cores
     # decode: a subset of sequences, each over its full kept cache
     nb = max(1, min(w.B, 2))

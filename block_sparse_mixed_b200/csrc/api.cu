@@ -274,21 +274,34 @@ size_t tria_prefill_workspace_bytes(const tria_dims* dims) {
   return prefill_layout(*dims).total;
 }
 
-int tria_prefill(const void* Q, const tria_kv_cache* cache, const tria_dims* dims, const int32_t* hi,
-                 const int32_t* keep, void* O, float* LSE, void* workspace, size_t workspace_bytes, void* stream) {
+namespace {
+
+// Checks shared by the prefill calls; on success fills the layout and device facts.
+int prefill_checks(const tria_kv_cache* cache, const tria_dims* dims, void* workspace, size_t workspace_bytes,
+                   PrefillLayout* L, DeviceInfo* dev) {
   int s = check_dims(dims);
   if (s != TRIA_OK) return s;
   if ((s = check_cache(cache)) != TRIA_OK) return s;
-  const tria_dims d = *dims;
+  const tria_dims& d = *dims;
   if (cache->B != d.B || cache->Hkv != d.Hkv || cache->D != d.D || cache->T != d.T || cache->capacity < d.S)
     return TRIA_ERR_INVALID_ARG;
-  if ((s = check_policy(hi, keep, d.Hq)) != TRIA_OK) return s;
-  if (Q == nullptr || O == nullptr || LSE == nullptr || !aligned16(Q) || !aligned16(O) || !aligned16(LSE))
-    return TRIA_ERR_INVALID_ARG;
-  const PrefillLayout L = prefill_layout(d);
-  if (workspace == nullptr || !aligned256(workspace) || workspace_bytes < L.total) return TRIA_ERR_WORKSPACE;
-  const DeviceInfo dev = device_info();
-  if (!dev.ok) return TRIA_ERR_UNSUPPORTED;
+  *L = prefill_layout(d);
+  if (workspace == nullptr || !aligned256(workspace) || workspace_bytes < L->total) return TRIA_ERR_WORKSPACE;
+  *dev = device_info();
+  if (!dev->ok) return TRIA_ERR_UNSUPPORTED;
+  return TRIA_OK;
+}
+
+}  // namespace
+
+int tria_prefill_prepare(const void* Q, const tria_kv_cache* cache, const tria_dims* dims, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  PrefillLayout L;
+  DeviceInfo dev;
+  int s = prefill_checks(cache, dims, workspace, workspace_bytes, &L, &dev);
+  if (s != TRIA_OK) return s;
+  if (Q == nullptr || !aligned16(Q)) return TRIA_ERR_INVALID_ARG;
+  const tria_dims d = *dims;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const int nb = d.S / d.T;
@@ -316,7 +329,23 @@ int tria_prefill(const void* Q, const tria_kv_cache* cache, const tria_dims* dim
   pa.vt4 = reinterpret_cast<__nv_bfloat16*>(ws + L.vt4);
   pa.cap = cache->capacity; pa.S = d.S; pa.nb = nb;
   if (launch_prepare(pa, d.D, d.T, groups, nb, st) != cudaSuccess) return TRIA_ERR_CUDA;
+  return TRIA_OK;
+}
 
+int tria_prefill_attend(const tria_kv_cache* cache, const tria_dims* dims, const int32_t* hi, const int32_t* keep,
+                        void* O, float* LSE, void* workspace, size_t workspace_bytes, void* stream) {
+  PrefillLayout L;
+  DeviceInfo dev;
+  int s = prefill_checks(cache, dims, workspace, workspace_bytes, &L, &dev);
+  if (s != TRIA_OK) return s;
+  const tria_dims d = *dims;
+  if ((s = check_policy(hi, keep, d.Hq)) != TRIA_OK) return s;
+  if (O == nullptr || LSE == nullptr || !aligned16(O) || !aligned16(LSE)) return TRIA_ERR_INVALID_ARG;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int nb = d.S / d.T;
+  const int64_t qrows = static_cast<int64_t>(d.B) * d.Hq * d.S;
+  const int groups = d.B * d.Hkv;
   // 3. the fused kernel
   PrefillMaps maps;
   const uint64_t krows = static_cast<uint64_t>(groups) * d.S;
@@ -351,6 +380,16 @@ int tria_prefill(const void* Q, const tria_kv_cache* cache, const tria_dims* dim
   a.err = reinterpret_cast<int*>(ws + L.ctrl);
   for (int h = 0; h < d.Hq; ++h) { a.hi[h] = hi[h]; a.keep[h] = keep[h]; }
   return cuda_status(launch_prefill(a, maps, d.D, d.T, dev.sms, st));
+}
+
+int tria_prefill(const void* Q, const tria_kv_cache* cache, const tria_dims* dims, const int32_t* hi,
+                 const int32_t* keep, void* O, float* LSE, void* workspace, size_t workspace_bytes, void* stream) {
+  // arguments of the second call are checked before the first one runs
+  int s = check_policy(hi, keep, dims != nullptr ? dims->Hq : 0);
+  if (dims == nullptr || s != TRIA_OK) return dims == nullptr ? TRIA_ERR_INVALID_ARG : s;
+  if (O == nullptr || LSE == nullptr || !aligned16(O) || !aligned16(LSE)) return TRIA_ERR_INVALID_ARG;
+  if ((s = tria_prefill_prepare(Q, cache, dims, workspace, workspace_bytes, stream)) != TRIA_OK) return s;
+  return tria_prefill_attend(cache, dims, hi, keep, O, LSE, workspace, workspace_bytes, stream);
 }
 
 size_t tria_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int T, int capacity) {

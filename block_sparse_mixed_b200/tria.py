@@ -69,6 +69,11 @@ def lib():
         L.tria_prefill.argtypes = [P, ctypes.POINTER(tria_kv_cache), ctypes.POINTER(tria_dims), P, P, P, P, P,
                                    SZ, P]
         L.tria_prefill.restype = I
+        L.tria_prefill_prepare.argtypes = [P, ctypes.POINTER(tria_kv_cache), ctypes.POINTER(tria_dims), P, SZ, P]
+        L.tria_prefill_prepare.restype = I
+        L.tria_prefill_attend.argtypes = [ctypes.POINTER(tria_kv_cache), ctypes.POINTER(tria_dims), P, P, P, P, P,
+                                          SZ, P]
+        L.tria_prefill_attend.restype = I
         L.tria_decode_workspace_bytes.argtypes = [I, I, I, I, I, I]
         L.tria_decode_workspace_bytes.restype = SZ
         L.tria_decode.argtypes = [P, ctypes.POINTER(tria_kv_cache), P, I, P, P, P, P, P, SZ, P]
@@ -188,6 +193,28 @@ def tria_prefill(Q: torch.Tensor, cache: CompressedKVCache, hi, keep, workspace:
     hi_a, keep_a = _host_i32(hi), _host_i32(keep)
     _check("tria_prefill", lib().tria_prefill(
         _dev_ptr(Q), ctypes.byref(cache.struct), ctypes.byref(dims), hi_a.ctypes.data_as(ctypes.c_void_p),
+        keep_a.ctypes.data_as(ctypes.c_void_p), _dev_ptr(O), _dev_ptr(LSE), _dev_ptr(workspace),
+        workspace.numel(), _stream(stream)))
+    return O, LSE
+
+
+def tria_prefill_prepare(Q: torch.Tensor, cache: CompressedKVCache, workspace: torch.Tensor, stream=None):
+    """First half of tria_prefill: Q codec and operand tiles into `workspace`."""
+    B, Hq, S, D = Q.shape
+    dims = tria_dims(B, Hq, cache.Hkv, S, D, cache.T)
+    _check("tria_prefill_prepare", lib().tria_prefill_prepare(
+        _dev_ptr(Q), ctypes.byref(cache.struct), ctypes.byref(dims), _dev_ptr(workspace), workspace.numel(),
+        _stream(stream)))
+
+
+def tria_prefill_attend(cache: CompressedKVCache, hi, keep, workspace: torch.Tensor, O: torch.Tensor,
+                        LSE: torch.Tensor, stream=None):
+    """Second half of tria_prefill: the fused kernel over a prepared workspace; writes O and LSE."""
+    B, Hq, S, D = O.shape
+    dims = tria_dims(B, Hq, cache.Hkv, S, D, cache.T)
+    hi_a, keep_a = _host_i32(hi), _host_i32(keep)
+    _check("tria_prefill_attend", lib().tria_prefill_attend(
+        ctypes.byref(cache.struct), ctypes.byref(dims), hi_a.ctypes.data_as(ctypes.c_void_p),
         keep_a.ctypes.data_as(ctypes.c_void_p), _dev_ptr(O), _dev_ptr(LSE), _dev_ptr(workspace),
         workspace.numel(), _stream(stream)))
     return O, LSE

@@ -130,6 +130,20 @@ int tria_prefill(const void* Q, const tria_kv_cache* cache, const tria_dims* dim
                  const int32_t* hi, const int32_t* keep, void* O, float* LSE,
                  void* workspace, size_t workspace_bytes, void* stream);
 
+/* The two halves of tria_prefill, for callers that time or schedule them apart.
+ * tria_prefill_prepare: Q codec (both planes) and the operand tiles built from
+ * the cache (4-bit K expanded to one code per byte, V dequantised to bf16 and
+ * transposed per block) into `workspace`; reads Q and the cache only.
+ * tria_prefill_attend: the fused block-sparse kernel over what prepare left in
+ * the same workspace, for the same cache and dims; writes O and LSE.
+ * prepare followed by attend on one stream equals tria_prefill. Arguments,
+ * layouts and errors are those of tria_prefill. */
+int tria_prefill_prepare(const void* Q, const tria_kv_cache* cache, const tria_dims* dims, void* workspace,
+                         size_t workspace_bytes, void* stream);
+int tria_prefill_attend(const tria_kv_cache* cache, const tria_dims* dims, const int32_t* hi,
+                        const int32_t* keep, void* O, float* LSE, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
 /* Workspace bytes tria_decode needs (0 if the arguments are invalid). */
 size_t tria_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int T, int capacity);
 

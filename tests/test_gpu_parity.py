@@ -243,3 +243,21 @@ def test_decode_equals_last_prefill_row(T):
     torch.cuda.synchronize()
     assert (Od.float() - O[:, :, S - 1].float()).abs().max().item() <= 1e-2
     assert (Ld - L[:, :, S - 1]).abs().max().item() <= 1e-3
+
+
+def test_prepare_then_attend_equals_prefill(T):
+    """tria_prefill_prepare + tria_prefill_attend on one stream give tria_prefill's bits."""
+    B, Hq, Hkv, S, D, Tb = 1, 4, 2, 1024, 128, 128
+    hi = np.array([1, 2, 0, 3], np.int32)
+    keep = np.array([3, 5, 2, 4], np.int32)
+    Q, K, V = seeded((B, Hq, S, D), 81, "cuda"), seeded((B, Hkv, S, D), 82, "cuda"), seeded((B, Hkv, S, D), 83, "cuda")
+    cache = T.CompressedKVCache(B, Hkv, D, Tb, S)
+    T.tria_quantize_kv(K, V, cache)
+    ws = torch.empty(T.tria_prefill_workspace_bytes(B, Hq, Hkv, S, D, Tb), dtype=torch.uint8, device="cuda")
+    O1, L1 = T.tria_prefill(Q, cache, hi, keep, workspace=ws)
+    O2, L2 = torch.empty_like(O1), torch.empty_like(L1)
+    T.tria_prefill_prepare(Q, cache, ws)
+    T.tria_prefill_attend(cache, hi, keep, ws, O2, L2)
+    torch.cuda.synchronize()
+    assert T.tria_workspace_status(ws) == 0
+    assert torch.equal(O1, O2) and torch.equal(L1, L2)
