@@ -48,6 +48,34 @@ def test_codec_bit_exact(T, oracle_mod):
         assert np.array_equal(c4.cpu().numpy(), oracle_mod.pack_int4(r4))
 
 
+def test_codec_ties_and_scales_bit_exact(T, oracle_mod):
+    """Rows whose 8-bit quotients sit exactly on half-integers at many binary scales
+    (amax = 127 * 2^e, so s8 = 2^e and x = (k + 1/2) 2^e), and a million random rows
+    spread over 2^-40 .. 2^40 in magnitude: codes and scales bit for bit."""
+    D = 64
+    ties = []
+    for e in range(-30, 31, 3):
+        for k0 in range(0, 126, 63):
+            row = torch.zeros(D)
+            row[0] = 127.0 * 2.0 ** e
+            ks = torch.arange(k0, k0 + D - 1) % 127
+            row[1:] = (ks.float() + 0.5) * 2.0 ** e * torch.where(ks % 2 == 0, 1.0, -1.0)
+            ties.append(row)
+    ties32 = torch.stack(ties)
+    ties = ties32.to(torch.bfloat16)
+    assert torch.equal(ties.float(), ties32)   # bf16 holds every tie exactly
+    g = torch.Generator().manual_seed(123)
+    rnd = torch.randn((1 << 20, D), generator=g)
+    rnd = rnd * torch.pow(2.0, torch.randint(-40, 41, (1 << 20, 1), generator=g).float())
+    x = torch.cat([ties, rnd.to(torch.bfloat16)])
+    c8, s8, c4, s4 = T.tria_quantize_rows(x.cuda())
+    r8, rs8, r4, rs4 = oracle_mod.quantize_rows(x, D)
+    assert np.array_equal(s8.cpu().numpy().view(np.uint32), rs8.view(np.uint32))
+    assert np.array_equal(s4.cpu().numpy().view(np.uint32), rs4.view(np.uint32))
+    assert np.array_equal(c8.cpu().numpy(), r8)
+    assert np.array_equal(c4.cpu().numpy(), oracle_mod.pack_int4(r4))
+
+
 def test_cache_write_and_append_bit_exact(T, oracle_mod):
     B, Hkv, D, Tb, cap = 2, 3, 128, 64, 320
     cache = T.CompressedKVCache(B, Hkv, D, Tb, cap)
