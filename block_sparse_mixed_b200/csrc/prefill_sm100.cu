@@ -53,7 +53,7 @@ constexpr int kMmaWarp = 17;
 // 4 x 128 x 104 + 128 x 64 = 61,440, within the launch total.
 constexpr int kRegsSoftmax = 104;
 constexpr int kRegsOther = 64;
-constexpr int kSlots = 2;               // S buffers in TMEM, one per pair
+constexpr int kPairs = 2;               // softmax pairs = O accumulators in TMEM
 constexpr int kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;    // raise the running max only past this growth
 
@@ -68,7 +68,12 @@ struct Cfg {
   static constexpr int kVTile = D * T * 2;                   // all V sub-tiles of a stage
   static constexpr int kStageRaw = kKTile + kVTile + T * 4;  // + K scales
   static constexpr int kStage = (kStageRaw + 1023) / 1024 * 1024;
-  static constexpr int kStages = T == 128 ? 3 : 4;
+  static constexpr int kStages = T == 128 ? 3 : 6;
+  // S buffers in TMEM (T columns each, below the O accumulators at 256): two at
+  // T = 128; four at T = 64, so that each pair has a second S ready while it
+  // works on one, and QK runs kLead loads ahead of P.V.
+  static constexpr int kSlots = T == 128 ? 2 : 4;
+  static constexpr int kLead = kSlots / 2;
   static constexpr int kQTile = kRows * kQKRowBytes;
   static constexpr int kOffQ8 = 0;
   static constexpr int kOffQ4 = kQTile;
@@ -87,9 +92,10 @@ struct Cfg {
 
 struct Bars {
   uint64_t q_full, q_empty, fin;
-  uint64_t o_done[kSlots];      // P.V of load g completes phase g/2 of o_done[g % 2]
-  uint64_t kv_full[4], kv_empty[4];
-  uint64_t s_full[kSlots], s_free[kSlots], p_full[kSlots];
+  uint64_t o_done[kPairs];      // P.V of load g completes phase g/2 of o_done[g % 2]
+  uint64_t o_fin;               // every P.V of the CTA's u-th tile: phase u
+  uint64_t kv_full[6], kv_empty[6];
+  uint64_t s_full[4], s_free[4], p_full[4];
   uint32_t tmem_base;
   int abort;
 };
@@ -264,8 +270,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
     }
-    for (int s = 0; s < kSlots; ++s) {
-      mbar_init(&bars->o_done[s], 1);
+    for (int p = 0; p < kPairs; ++p) mbar_init(&bars->o_done[p], 1);
+    mbar_init(&bars->o_fin, 1);
+    for (int s = 0; s < C::kSlots; ++s) {
       mbar_init(&bars->s_full[s], 1);
       mbar_init(&bars->s_free[s], 1);
       mbar_init(&bars->p_full[s], kPairThreads);
@@ -354,17 +361,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t q8a = smem_u32(sQ8), q4a = smem_u32(sQ4);
       // P.V of load gg into the O accumulator of its parity; `first` overwrites.
       auto pv = [&](uint32_t gg, bool first) -> bool {
-        const int st = gg % C::kStages, sl = gg % kSlots;
+        const int st = gg % C::kStages, sl = gg % C::kSlots, acc = gg % kPairs;
         const uint32_t vbase = smem_u32(sV(st));
-        if (!warp_wait(&bars->p_full[sl], (gg / kSlots) & 1)) return false;
+        if (!warp_wait(&bars->p_full[sl], (gg / C::kSlots) & 1)) return false;
         tc_fence_after();
         if (elect_one()) {
 #pragma unroll
           for (int s = 0; s < T / 16; ++s) {
             const uint64_t bdesc = sw128_desc(vbase + (s / 4) * C::kVSub + (s % 4) * 32);
-            mma_bf16_ts(tmem + o_col(sl), tmem + sl * T + s * 8, bdesc, C::kIdescPV, (first && s == 0) ? 0u : 1u);
+            mma_bf16_ts(tmem + o_col(acc), tmem + sl * T + s * 8, bdesc, C::kIdescPV, (first && s == 0) ? 0u : 1u);
           }
-          mma_commit(&bars->o_done[sl]);
+          mma_commit(&bars->o_done[acc]);
           mma_commit(&bars->kv_empty[st]);
           mma_commit(&bars->s_free[sl]);
         }
@@ -378,16 +385,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         LoadSeq seq;
         seq.init(u.i0, u.nq, a.hi[u.hq], a.keep[u.hq]);
         int j, plane, l = 0;
-        bool used[kSlots] = {false, false};   // accumulator written in this tile yet?
+        bool used[kPairs] = {false, false};   // accumulator written in this tile yet?
         auto pv_next = [&](uint32_t gg) -> bool {
-          const bool first = !used[gg % kSlots];
-          used[gg % kSlots] = true;
+          const bool first = !used[gg % kPairs];
+          used[gg % kPairs] = true;
           return pv(gg, first);
         };
+        // order: QK(g), then P.V(g - kLead): QK runs kLead loads ahead
         while (seq.next(j, plane)) {
-          const int st = g % C::kStages, sl = g % kSlots;
+          const int st = g % C::kStages, sl = g % C::kSlots;
           if (!(ok = warp_wait(&bars->kv_full[st], (g / C::kStages) & 1))) break;
-          if (g >= static_cast<uint32_t>(kSlots) && !(ok = warp_wait(&bars->s_free[sl], ((g / kSlots) - 1) & 1)))
+          if (g >= static_cast<uint32_t>(C::kSlots) &&
+              !(ok = warp_wait(&bars->s_free[sl], ((g / C::kSlots) - 1) & 1)))
             break;
           tc_fence_after();
           const uint32_t abase = plane == 8 ? q8a : q4a;
@@ -400,13 +409,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(&bars->s_full[sl]);
           }
           __syncwarp();
-          if (l > 0 && !(ok = pv_next(g - 1))) break;
+          if (l >= C::kLead && !(ok = pv_next(g - C::kLead))) break;
           ++l;
           ++g;
         }
         if (!ok) break;
-        if (l > 0 && !(ok = pv_next(g - 1))) break;
-        if (elect_one()) mma_commit(&bars->q_empty);
+        for (int k = (l < C::kLead ? l : C::kLead); k > 0 && ok; --k) ok = pv_next(g - k);
+        if (!ok) break;
+        if (elect_one()) {
+          mma_commit(&bars->q_empty);
+          mma_commit(&bars->o_fin);
+        }
         __syncwarp();
       }
       // wait for every tensor-core op this CTA issued before TMEM is released
@@ -423,8 +436,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int sub = warp % 4;                 // TMEM lane quarter
     const int row = sub * 32 + lane;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(sub * 32) << 16);
-    const uint32_t my_s = lane_addr + pair * T + half * TH;          // S columns of my keys
-    const uint32_t my_p = lane_addr + pair * T + half * (TH / 2);    // P words of my keys
+    const uint32_t my_s = lane_addr + half * TH;                     // + slot * T: S columns of my keys
+    const uint32_t my_p = lane_addr + half * (TH / 2);               // + slot * T: P words of my keys
     const uint32_t my_o = lane_addr + o_col(pair) + half * (D / 2);  // O columns rescaled here
     const uint32_t pair_bar = 1 + pair * 4 + sub;                    // 64 threads: this row's pair
     const uint32_t row_bar = 9 + sub;                                // 128 threads: all four of the row
@@ -449,20 +462,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       seq.init(u.i0, u.nq, hi, keep);
       int j, plane;
       while (seq.next(j, plane)) {
-        if (static_cast<int>(g % kSlots) != pair) { ++g; continue; }
-        const int st = g % C::kStages;
+        if (static_cast<int>(g % kPairs) != pair) { ++g; continue; }
+        const int st = g % C::kStages, sl = g % C::kSlots;
+        const uint32_t slot_col = static_cast<uint32_t>(sl * T);
         if (!(ok = mbar_wait(&bars->kv_full[st], (g / C::kStages) & 1, abort, a.err))) break;
-        if (!(ok = mbar_wait(&bars->s_full[pair], (g / kSlots) & 1, abort, a.err))) break;
-        // QK of this load waited for the P.V two loads back, which used this slot and
-        // this accumulator: the accumulator is final for now and may be rescaled.
+        if (!(ok = mbar_wait(&bars->s_full[sl], (g / C::kSlots) & 1, abort, a.err))) break;
         tc_fence_after();
+        const bool had_prev = g_mine >= 0;        // this pair's previous load (g - 2) is in this tile
         g_mine = g;
         const int act = valid ? tile_action(ir, j, hi, keep) : ACT_NONE;   // uniform over the warp pair
         if (act == plane) {
           const int kmax = (j == ir) ? rl - half * TH : TH;   // my keys [0, kmax] are visible
           uint32_t r[TH];
 #pragma unroll
-          for (int c = 0; c < TH / 32; ++c) tmem_ld32(my_s + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+          for (int c = 0; c < TH / 32; ++c)
+            tmem_ld32(my_s + slot_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
           const float* sk = sScale(st) + half * TH;
           const float alpha = plane == 8 ? a8 : a4;
           tmem_wait_ld();
@@ -487,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t pk[TH / 2];
             if (masked) probs<TH, true>(y, al2, nm2, kmax, pk, acc);
             else probs<TH, false>(y, al2, nm2, kmax, pk, acc);
-            tmem_store_words<TH / 2>(my_p, pk);
+            tmem_store_words<TH / 2>(my_p + slot_col, pk);
           }
           float s0, s1;
           up2(add2(add2(acc[0], acc[1]), add2(acc[2], acc[3])), s0, s1);
@@ -496,6 +510,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           // may start). TMEM loads/stores are warp-collective: the whole warp takes part
           // when any lane must, lanes that need not using the factor 1.
           if (__any_sync(0xffffffffu, rescale_o)) {
+            // P.V of this pair's previous load (g - 2) writes this accumulator: it
+            // must be complete. With kLead = 1 the completed QK of this load implies
+            // it; with kLead = 2 it may still run, and o_done[pair] is then at most
+            // one phase short of it (P.V of this load is not issued yet).
+            if (C::kLead > 1 && had_prev &&
+                !(ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[pair], ((g - 2) / kPairs) & 1, abort, a.err))))
+              break;
+            tc_fence_after();
 #pragma unroll
             for (int c = 0; c < D / 64; ++c) {
               uint32_t o[32];
@@ -510,21 +532,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t z[TH / 2];
 #pragma unroll
           for (int k = 0; k < TH / 2; ++k) z[k] = 0u;
-          tmem_store_words<TH / 2>(my_p, z);
+          tmem_store_words<TH / 2>(my_p + slot_col, z);
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars->p_full[pair]);
+        mbar_arrive(&bars->p_full[sl]);
         ++g;
       }
       if (!ok) break;
-      // Epilogue. The last P.V into this pair's accumulator: its QK was seen, so the
-      // P.V two loads earlier is complete and o_done[pair] is at most one phase short.
-      if (g_mine >= 0) {
-        const uint32_t gm = static_cast<uint32_t>(g_mine);
-        if (!(ok = mbar_wait(&bars->o_done[pair], (gm / kSlots) & 1, abort, a.err))) break;
-        tc_fence_after();
-      }
+      // Epilogue: every P.V of this tile has completed (o_fin, one phase per tile; the
+      // next tile's first P.V needs a P from after this epilogue, so the barrier is at
+      // most one phase short).
+      if (!(ok = mbar_wait(&bars->o_fin, uloc & 1, abort, a.err))) break;
+      tc_fence_after();
       float* xe = xepi + (uloc & 1) * (2 * 2 * 2 * 128);
       auto slot = [&](int p, int h, int v) { return xe + ((p * 2 + h) * 2 + v) * 128 + row; };
       *slot(pair, half, 0) = m_run;
