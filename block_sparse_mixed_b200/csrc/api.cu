@@ -378,7 +378,9 @@ int tria_prefill_attend(const tria_kv_cache* cache, const tria_dims* dims, const
   a.k8s = cache->k8_scale; a.k4s = cache->k4_scale;
   a.O = static_cast<__nv_bfloat16*>(O); a.LSE = LSE;
   a.err = reinterpret_cast<int*>(ws + L.ctrl);
+  a.work = reinterpret_cast<int*>(ws + L.ctrl) + 4;
   for (int h = 0; h < d.Hq; ++h) { a.hi[h] = hi[h]; a.keep[h] = keep[h]; }
+  if (cudaMemsetAsync(a.work, 0, sizeof(int), st) != cudaSuccess) return TRIA_ERR_CUDA;   // tile counter
   return cuda_status(launch_prefill(a, maps, d.D, d.T, dev.sms, st));
 }
 

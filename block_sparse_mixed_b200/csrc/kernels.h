@@ -60,6 +60,7 @@ struct PrefillArgs {
   __nv_bfloat16* O;
   float* LSE;
   int* err;
+  int* work;              // next query tile (dynamic scheduling); zero before the launch
   int hi[kMaxHeads];
   int keep[kMaxHeads];
 };

@@ -68,16 +68,18 @@ struct Cfg {
   static constexpr int kVTile = D * T * 2;                   // all V sub-tiles of a stage
   static constexpr int kStageRaw = kKTile + kVTile + T * 4;  // + K scales
   static constexpr int kStage = (kStageRaw + 1023) / 1024 * 1024;
-  static constexpr int kStages = T == 128 ? 3 : 6;
+  static constexpr int kStages = T == 128 ? 3 : 5;
   // S buffers in TMEM (T columns each, below the O accumulators at 256): two at
   // T = 128; four at T = 64, so that each pair has a second S ready while it
   // works on one, and QK runs kLead loads ahead of P.V.
   static constexpr int kSlots = T == 128 ? 2 : 4;
   static constexpr int kLead = kSlots / 2;
   static constexpr int kQTile = kRows * kQKRowBytes;
-  static constexpr int kOffQ8 = 0;
+  // Q codes of two tiles (both planes each): the next tile's Q is loaded while
+  // the current one is in use
+  static constexpr int kOffQ8 = 0;                           // + buffer * 2 * kQTile
   static constexpr int kOffQ4 = kQTile;
-  static constexpr int kOffStage = 2 * kQTile;
+  static constexpr int kOffStage = 4 * kQTile;
   static constexpr int kOffBar = kOffStage + kStages * kStage;
   static constexpr int kOffX = kOffBar + 1024;               // row-max and epilogue exchanges
   static constexpr int kXBytes = 2 * 2 * 128 * 4 + 2 * 2 * 2 * 2 * 128 * 4;   // 2 KB + 8 KB
@@ -90,14 +92,28 @@ struct Cfg {
   static constexpr uint32_t kIdescPV = idesc_bf16(kRows, D);
 };
 
+constexpr int kUnitRing = 8;            // tiles published ahead of the consumers
+
 struct Bars {
-  uint64_t q_full, q_empty, fin;
-  uint64_t o_done[kPairs];      // P.V of load g completes phase g/2 of o_done[g % 2]
+  uint64_t q_full[2], q_empty[2], fin;  // Q buffer b holds the CTA's tiles u with u % 2 == b
   uint64_t o_fin;               // every P.V of the CTA's u-th tile: phase u
+  // kv_empty[st] completes when the P.V of the load in stage st completes: it also
+  // tells the MMA warp that the S slot of that load is free, and the softmax that
+  // the O accumulator it wrote may be rescaled
   uint64_t kv_full[6], kv_empty[6];
-  uint64_t s_full[4], s_free[4], p_full[4];
+  uint64_t s_full[4], p_full[4];
   uint32_t tmem_base;
   int abort;
+  // Published by the producer so that no other role walks the load sequence:
+  // per stage, the load's key block and plane (kLastLoad marks a tile's last
+  // load), visible after kv_full; per tile u of this CTA, the tile's index and
+  // load count in ring entry u % kUnitRing (index -1: no more tiles), visible
+  // after phase u / kUnitRing of unit_ready[u % kUnitRing]. The ring cannot be
+  // lapped: a tile has at least one load, and the producer runs at most kStages
+  // loads ahead of the P.V that needs the slowest softmax pair.
+  int2 info[6];
+  int unit_w[kUnitRing], unit_loads[kUnitRing];
+  uint64_t unit_ready[kUnitRing];
 };
 
 // The (key block, plane) loads of one query tile, in ascending key-block order;
@@ -129,6 +145,8 @@ struct LoadSeq {
     return false;
   }
 };
+
+constexpr int kLastLoad = 1 << 8;       // flag in info[].y next to the plane
 
 struct Unit {
   int b, hq, kvh, i0, nq;
@@ -263,18 +281,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x % 32;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
-    mbar_init(&bars->q_empty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->q_full[b], 1);
+      mbar_init(&bars->q_empty[b], 1);
+    }
     mbar_init(&bars->fin, 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
     }
-    for (int p = 0; p < kPairs; ++p) mbar_init(&bars->o_done[p], 1);
     mbar_init(&bars->o_fin, 1);
+    for (int r = 0; r < kUnitRing; ++r) mbar_init(&bars->unit_ready[r], 1);
     for (int s = 0; s < C::kSlots; ++s) {
       mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->s_free[s], 1);
       mbar_init(&bars->p_full[s], kPairThreads);
     }
     bars->abort = 0;
@@ -292,7 +311,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = bars->tmem_base;
+  // One CTA per SM allocates all 512 columns, so the allocation starts at lane 0,
+  // column 0; TMEM addresses below are then compile-time constants plus uniform
+  // offsets. A different base is reported as an error and the CTA does no work.
+  constexpr uint32_t tmem = 0;
+  if (bars->tmem_base != 0) {
+    if (threadIdx.x == 0) atomicExch(a.err, TRIA_ERR_BOUNDS);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+      tc_fence_after();
+      tmem_dealloc(bars->tmem_base, kTmemCols);
+    }
+    return;
+  }
 
   uint8_t* sQ8 = smem + C::kOffQ8;
   uint8_t* sQ4 = smem + C::kOffQ4;
@@ -312,32 +344,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     if (warp == kProducerWarp) {
       // ---------------------------------------------------------- producer
-      uint32_t g = 0, uloc = 0, q_issued = 0;
+      uint32_t g = 0, uloc = 0;
       bool ok = true;
-      for (int w = blockIdx.x; w < a.n_units && ok; w += gridDim.x, ++uloc) {
+      for (;; ++uloc) {
+        // next tile from the kernel-wide counter (longest tiles first, see unit_of)
+        int w = 0;
+        if (lane == 0) w = atomicAdd(a.work, 1);
+        w = __shfl_sync(0xffffffffu, w, 0);
+        const int r = uloc % kUnitRing;
+        if (w >= a.n_units) {
+          if (elect_one()) {
+            bars->unit_w[r] = -1;
+            mbar_arrive(&bars->unit_ready[r]);
+          }
+          __syncwarp();
+          break;
+        }
         const Unit u = unit_of(a, w, C::kQBlocks);
-        if (uloc > 0 && !(ok = warp_wait(&bars->q_empty, (uloc - 1) & 1))) break;
-        ++q_issued;
+        int n_loads = 0;
+        {
+          LoadSeq cnt;
+          cnt.init(u.i0, u.nq, a.hi[u.hq], a.keep[u.hq]);
+          int jj, pp;
+          while (cnt.next(jj, pp)) ++n_loads;
+        }
+        // Q buffer uloc % 2 is free once the QKs of this CTA's tile uloc - 2 are done
+        const int qb = uloc & 1;
+        if (uloc >= 2 && !(ok = warp_wait(&bars->q_empty[qb], ((uloc >> 1) - 1) & 1))) break;
         const int qrow = (u.b * a.Hq + u.hq) * a.S + u.i0 * T;
         if (elect_one()) {
-          mbar_arrive_expect_tx(&bars->q_full, 2 * C::kQTile);
-          tma_load_2d(sQ8, &maps.q8, &bars->q_full, 0, qrow);
-          tma_load_2d(sQ4, &maps.q4, &bars->q_full, 0, qrow);
+          bars->unit_w[r] = w;
+          bars->unit_loads[r] = n_loads;
+          mbar_arrive(&bars->unit_ready[r]);   // release: the entry is visible after the wait
+          mbar_arrive_expect_tx(&bars->q_full[qb], 2 * C::kQTile);
+          tma_load_2d(sQ8 + qb * 2 * C::kQTile, &maps.q8, &bars->q_full[qb], 0, qrow);
+          tma_load_2d(sQ4 + qb * 2 * C::kQTile, &maps.q4, &bars->q_full[qb], 0, qrow);
         }
         __syncwarp();
         LoadSeq seq;
         seq.init(u.i0, u.nq, a.hi[u.hq], a.keep[u.hq]);
         const int64_t grp = static_cast<int64_t>(u.b) * a.Hkv + u.kvh;
-        int j, plane;
+        int j, plane, k_load = 0;
         while (seq.next(j, plane)) {
           const int st = g % C::kStages;
           if (g >= static_cast<uint32_t>(C::kStages) && !(ok = warp_wait(&bars->kv_empty[st], ((g / C::kStages) - 1) & 1)))
             break;
+          ++k_load;
           const int krow = static_cast<int>(grp * (plane == 8 ? a.cap8 : static_cast<int64_t>(a.S)) +
                                             static_cast<int64_t>(j) * T);
           const int vrow = static_cast<int>((grp * a.nb + j) * D);
           const float* ks = (plane == 8 ? a.k8s : a.k4s) + grp * a.cap + static_cast<int64_t>(j) * T;
           if (elect_one()) {
+            bars->info[st] = make_int2(j, plane | (k_load == n_loads ? kLastLoad : 0));   // released by the arrive
             mbar_arrive_expect_tx(&bars->kv_full[st], C::kStageTx);
             tma_load_2d(sK(st), plane == 8 ? &maps.k8 : &maps.k4, &bars->kv_full[st], 0, krow);
 #pragma unroll
@@ -349,11 +407,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           ++g;
         }
+        if (!ok) break;
       }
       // let every copy this CTA issued land before the block exits
       for (uint32_t k = (g > static_cast<uint32_t>(C::kStages) ? g - C::kStages : 0); k < g; ++k)
         drain_wait(&bars->kv_full[k % C::kStages], (k / C::kStages) & 1);
-      if (q_issued > 0) drain_wait(&bars->q_full, (q_issued - 1) & 1);
+      for (uint32_t k = (uloc > 2 ? uloc - 2 : 0); k < uloc; ++k) drain_wait(&bars->q_full[k & 1], (k >> 1) & 1);
     } else if (warp == kMmaWarp) {
       // ---------------------------------------------------------- MMA issuer
       uint32_t g = 0, uloc = 0;
@@ -365,26 +424,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t vbase = smem_u32(sV(st));
         if (!warp_wait(&bars->p_full[sl], (gg / C::kSlots) & 1)) return false;
         tc_fence_after();
+        const uint64_t vdesc = sw128_desc(vbase);
         if (elect_one()) {
 #pragma unroll
           for (int s = 0; s < T / 16; ++s) {
-            const uint64_t bdesc = sw128_desc(vbase + (s / 4) * C::kVSub + (s % 4) * 32);
+            // +((s / 4) * sub-tile + (s % 4) * 32 bytes) in the descriptor's 16-byte units
+            const uint64_t bdesc = vdesc + static_cast<uint64_t>(((s / 4) * C::kVSub + (s % 4) * 32) >> 4);
             mma_bf16_ts(tmem + o_col(acc), tmem + sl * T + s * 8, bdesc, C::kIdescPV, (first && s == 0) ? 0u : 1u);
           }
-          mma_commit(&bars->o_done[acc]);
           mma_commit(&bars->kv_empty[st]);
-          mma_commit(&bars->s_free[sl]);
         }
         __syncwarp();
         return true;
       };
-      for (int w = blockIdx.x; w < a.n_units && ok; w += gridDim.x, ++uloc) {
-        const Unit u = unit_of(a, w, C::kQBlocks);
-        if (!(ok = warp_wait(&bars->q_full, uloc & 1))) break;
+      for (;; ++uloc) {
+        const int r = uloc % kUnitRing;
+        if (!(ok = warp_wait(&bars->unit_ready[r], (uloc / kUnitRing) & 1))) break;
+        if (bars->unit_w[r] < 0) break;                 // no more tiles
+        const int qb = uloc & 1;
+        if (!(ok = warp_wait(&bars->q_full[qb], (uloc >> 1) & 1))) break;
         tc_fence_after();
-        LoadSeq seq;
-        seq.init(u.i0, u.nq, a.hi[u.hq], a.keep[u.hq]);
-        int j, plane, l = 0;
+        const uint32_t qoff = static_cast<uint32_t>(qb * 2 * C::kQTile);
+        int l = 0;
         bool used[kPairs] = {false, false};   // accumulator written in this tile yet?
         auto pv_next = [&](uint32_t gg) -> bool {
           const bool first = !used[gg % kPairs];
@@ -392,22 +453,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           return pv(gg, first);
         };
         // order: QK(g), then P.V(g - kLead): QK runs kLead loads ahead
-        while (seq.next(j, plane)) {
+        bool last = false;
+        while (!last) {
           const int st = g % C::kStages, sl = g % C::kSlots;
           if (!(ok = warp_wait(&bars->kv_full[st], (g / C::kStages) & 1))) break;
-          if (g >= static_cast<uint32_t>(C::kSlots) &&
-              !(ok = warp_wait(&bars->s_free[sl], ((g / C::kSlots) - 1) & 1)))
-            break;
+          const int2 inf = bars->info[st];
+          const int plane = inf.y & 0xff;
+          last = (inf.y & kLastLoad) != 0;
+          // the slot's previous S belonged to load g - kSlots: its P.V must be complete
+          if (g >= static_cast<uint32_t>(C::kSlots)) {
+            const uint32_t gp = g - C::kSlots;
+            if (!(ok = warp_wait(&bars->kv_empty[gp % C::kStages], (gp / C::kStages) & 1))) break;
+          }
           tc_fence_after();
-          const uint32_t abase = plane == 8 ? q8a : q4a;
+          const uint32_t abase = (plane == 8 ? q8a : q4a) + qoff;
           const uint32_t bbase = smem_u32(sK(st));
+          const uint64_t adesc = sw128_desc(abase), bdesc = sw128_desc(bbase);
           if (elect_one()) {
 #pragma unroll
-            for (int k = 0; k < kQKRowBytes / 32; ++k)
-              mma_i8_ss(tmem + sl * T, sw128_desc(abase + 32 * k), sw128_desc(bbase + 32 * k), C::kIdescQK,
-                        k > 0 ? 1u : 0u);
+            for (int k = 0; k < kQKRowBytes / 32; ++k)   // +32 bytes along K = +2 descriptor units
+              mma_i8_ss(tmem + sl * T, adesc + 2 * k, bdesc + 2 * k, C::kIdescQK, k > 0 ? 1u : 0u);
             mma_commit(&bars->s_full[sl]);
           }
+          __syncwarp();
+          // the tile's last QK has read its Q buffer: the producer may refill it
+          if (last && elect_one()) mma_commit(&bars->q_empty[qb]);
           __syncwarp();
           if (l >= C::kLead && !(ok = pv_next(g - C::kLead))) break;
           ++l;
@@ -416,10 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         for (int k = (l < C::kLead ? l : C::kLead); k > 0 && ok; --k) ok = pv_next(g - k);
         if (!ok) break;
-        if (elect_one()) {
-          mma_commit(&bars->q_empty);
-          mma_commit(&bars->o_fin);
-        }
+        if (elect_one()) mma_commit(&bars->o_fin);
         __syncwarp();
       }
       // wait for every tensor-core op this CTA issued before TMEM is released
@@ -446,7 +513,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* xepi = xmax + 2 * 2 * 128;
     uint32_t g = 0, uloc = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < a.n_units && ok; w += gridDim.x, ++uloc) {
+    for (;; ++uloc) {
+      // the CTA's next tile and its load count, published by the producer
+      const int r = uloc % kUnitRing;
+      if (!(ok = mbar_wait(&bars->unit_ready[r], (uloc / kUnitRing) & 1, abort, a.err))) break;
+      const int w = bars->unit_w[r];
+      if (w < 0) break;                                 // no more tiles
       const Unit u = unit_of(a, w, C::kQBlocks);
       const int qb = row / T;
       const int rl = row % T;
@@ -458,16 +530,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int hi = a.hi[u.hq], keep = a.keep[u.hq];
       float m_run = -INFINITY, l_run = 0.0f;     // m_run: shared by both halves of the pair
       int64_t g_mine = -1;                        // last load of this tile handled by this pair
-      LoadSeq seq;
-      seq.init(u.i0, u.nq, hi, keep);
-      int j, plane;
-      while (seq.next(j, plane)) {
-        if (static_cast<int>(g % kPairs) != pair) { ++g; continue; }
+      // this tile's loads are g0 .. g0 + n - 1 in the CTA's order; the pair takes
+      // those of its parity
+      const uint32_t g0 = g, g_end = g0 + static_cast<uint32_t>(bars->unit_loads[r]);
+      for (g = g0 + ((g0 % kPairs) == static_cast<uint32_t>(pair) ? 0u : 1u); g < g_end; g += kPairs) {
         const int st = g % C::kStages, sl = g % C::kSlots;
         const uint32_t slot_col = static_cast<uint32_t>(sl * T);
         if (!(ok = mbar_wait(&bars->kv_full[st], (g / C::kStages) & 1, abort, a.err))) break;
         if (!(ok = mbar_wait(&bars->s_full[sl], (g / C::kSlots) & 1, abort, a.err))) break;
         tc_fence_after();
+        const int2 inf = bars->info[st];
+        const int j = inf.x, plane = inf.y & 0xff;
         const bool had_prev = g_mine >= 0;        // this pair's previous load (g - 2) is in this tile
         g_mine = g;
         const int act = valid ? tile_action(ir, j, hi, keep) : ACT_NONE;   // uniform over the warp pair
@@ -512,11 +585,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (__any_sync(0xffffffffu, rescale_o)) {
             // P.V of this pair's previous load (g - 2) writes this accumulator: it
             // must be complete. With kLead = 1 the completed QK of this load implies
-            // it; with kLead = 2 it may still run, and o_done[pair] is then at most
-            // one phase short of it (P.V of this load is not issued yet).
-            if (C::kLead > 1 && had_prev &&
-                !(ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[pair], ((g - 2) / kPairs) & 1, abort, a.err))))
-              break;
+            // it; with kLead = 2 it may still run. Its stage's kv_empty is then at
+            // most one phase short of it: the stage's next load is g - 2 + kStages.
+            if (C::kLead > 1 && had_prev) {
+              const uint32_t gp = g - 2;
+              if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars->kv_empty[gp % C::kStages],
+                                                           (gp / C::kStages) & 1, abort, a.err))))
+                break;
+            }
             tc_fence_after();
 #pragma unroll
             for (int c = 0; c < D / 64; ++c) {
@@ -537,9 +613,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars->p_full[sl]);
-        ++g;
       }
       if (!ok) break;
+      g = g_end;
       // Epilogue: every P.V of this tile has completed (o_fin, one phase per tile; the
       // next tile's first P.V needs a P from after this epilogue, so the barrier is at
       // most one phase short).
