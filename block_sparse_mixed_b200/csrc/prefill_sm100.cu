@@ -60,19 +60,24 @@ constexpr float kRescaleLog2 = 8.0f;    // raise the running max only past this 
 // O accumulator of pair p: D columns at 256 + 128 p.
 __host__ __device__ constexpr uint32_t o_col(int p) { return p == 0 ? 256u : 384u; }
 
+// A load carries 128 keys: one key block at T = 128, two key blocks of the same
+// plane at T = 64 (the producer pairs them; a block left alone is loaded twice
+// and its second copy masked). The tensor-core side is the same for both.
+constexpr int kKeys = 128;
+
 template <int T, int D>
 struct Cfg {
   static constexpr int kQBlocks = kRows / T;                 // query blocks per tile
-  static constexpr int kKTile = T * kQKRowBytes;             // K codes per stage
+  static constexpr int kBlocksPerLoad = kKeys / T;           // key blocks per load
+  static constexpr int kKTile = kKeys * kQKRowBytes;         // K codes per stage
   static constexpr int kVSub = D * 128;                      // one V sub-tile: D rows x 64 keys
-  static constexpr int kVTile = D * T * 2;                   // all V sub-tiles of a stage
-  static constexpr int kStageRaw = kKTile + kVTile + T * 4;  // + K scales
+  static constexpr int kVTile = D * kKeys * 2;               // all V sub-tiles of a stage
+  static constexpr int kStageRaw = kKTile + kVTile + kKeys * 4;   // + K scales
   static constexpr int kStage = (kStageRaw + 1023) / 1024 * 1024;
-  static constexpr int kStages = T == 128 ? 3 : 5;
-  // S buffers in TMEM (T columns each, below the O accumulators at 256): two at
-  // T = 128; four at T = 64, so that each pair has a second S ready while it
-  // works on one, and QK runs kLead loads ahead of P.V.
-  static constexpr int kSlots = T == 128 ? 2 : 4;
+  static constexpr int kStages = 3;
+  // S buffers in TMEM (kKeys columns each, below the O accumulators at 256); QK
+  // of a load is issued before the P.V of the load before it.
+  static constexpr int kSlots = 2;
   static constexpr int kLead = kSlots / 2;
   static constexpr int kQTile = kRows * kQKRowBytes;
   // Q codes of two tiles (both planes each): the next tile's Q is loaded while
@@ -87,8 +92,8 @@ struct Cfg {
   // is resident per SM
   static constexpr int kSmemNeed = kOffX + kXBytes + 1024;
   static constexpr int kSmem = kSmemNeed > 120 * 1024 ? kSmemNeed : 120 * 1024;
-  static constexpr uint32_t kStageTx = kKTile + kVTile + T * 4;
-  static constexpr uint32_t kIdescQK = idesc_i8(kRows, T);
+  static constexpr uint32_t kStageTx = kKTile + kVTile + kKeys * 4;
+  static constexpr uint32_t kIdescQK = idesc_i8(kRows, kKeys);
   static constexpr uint32_t kIdescPV = idesc_bf16(kRows, D);
 };
 
@@ -111,7 +116,7 @@ struct Bars {
   // after phase u / kUnitRing of unit_ready[u % kUnitRing]. The ring cannot be
   // lapped: a tile has at least one load, and the producer runs at most kStages
   // loads ahead of the P.V that needs the slowest softmax pair.
-  int2 info[6];
+  int4 info[6];                 // (j0, j1, plane | kLastLoad, 0)
   int unit_w[kUnitRing], unit_loads[kUnitRing];
   uint64_t unit_ready[kUnitRing];
 };
@@ -146,7 +151,51 @@ struct LoadSeq {
   }
 };
 
-constexpr int kLastLoad = 1 << 8;       // flag in info[].y next to the plane
+constexpr int kLastLoad = 1 << 8;       // flag in info[].z next to the plane
+
+// The 128-key loads of a tile: with one key block per load (T = 128) the
+// (block, plane) pairs of LoadSeq, each as (j, j); with two (T = 64) consecutive
+// pairs of the same plane merged into (j0, j1), and a block whose neighbour in
+// the sequence has the other plane alone as (j0, -1).
+template <int BPL>
+struct LoadPairs {
+  LoadSeq seq;
+  int pj, pplane;
+  bool pending;
+  __device__ void init(int i0, int nq, int hi, int keep) {
+    seq.init(i0, nq, hi, keep);
+    pending = false;
+  }
+  __device__ bool next(int& j0, int& j1, int& plane) {
+    if constexpr (BPL == 1) {
+      if (!seq.next(j0, plane)) return false;
+      j1 = j0;
+      return true;
+    } else {
+      int j, pl;
+      while (seq.next(j, pl)) {
+        if (!pending) {
+          pj = j; pplane = pl; pending = true;
+          continue;
+        }
+        if (pl == pplane) {            // merge with the pending block
+          j0 = pj; j1 = j; plane = pl;
+          pending = false;
+          return true;
+        }
+        j0 = pj; j1 = -1; plane = pplane;   // emit the pending block alone
+        pj = j; pplane = pl;
+        return true;
+      }
+      if (pending) {
+        j0 = pj; j1 = -1; plane = pplane;
+        pending = false;
+        return true;
+      }
+      return false;
+    }
+  }
+};
 
 struct Unit {
   int b, hq, kvh, i0, nq;
@@ -363,10 +412,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Unit u = unit_of(a, w, C::kQBlocks);
         int n_loads = 0;
         {
-          LoadSeq cnt;
+          LoadPairs<C::kBlocksPerLoad> cnt;
           cnt.init(u.i0, u.nq, a.hi[u.hq], a.keep[u.hq]);
-          int jj, pp;
-          while (cnt.next(jj, pp)) ++n_loads;
+          int j0, j1, pp;
+          while (cnt.next(j0, j1, pp)) ++n_loads;
         }
         // Q buffer uloc % 2 is free once the QKs of this CTA's tile uloc - 2 are done
         const int qb = uloc & 1;
@@ -381,28 +430,40 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(sQ4 + qb * 2 * C::kQTile, &maps.q4, &bars->q_full[qb], 0, qrow);
         }
         __syncwarp();
-        LoadSeq seq;
+        LoadPairs<C::kBlocksPerLoad> seq;
         seq.init(u.i0, u.nq, a.hi[u.hq], a.keep[u.hq]);
         const int64_t grp = static_cast<int64_t>(u.b) * a.Hkv + u.kvh;
-        int j, plane, k_load = 0;
-        while (seq.next(j, plane)) {
+        int j0, j1, plane, k_load = 0;
+        while (seq.next(j0, j1, plane)) {
           const int st = g % C::kStages;
           if (g >= static_cast<uint32_t>(C::kStages) && !(ok = warp_wait(&bars->kv_empty[st], ((g / C::kStages) - 1) & 1)))
             break;
           ++k_load;
-          const int krow = static_cast<int>(grp * (plane == 8 ? a.cap8 : static_cast<int64_t>(a.S)) +
-                                            static_cast<int64_t>(j) * T);
-          const int vrow = static_cast<int>((grp * a.nb + j) * D);
-          const float* ks = (plane == 8 ? a.k8s : a.k4s) + grp * a.cap + static_cast<int64_t>(j) * T;
+          const CUtensorMap* kmap = plane == 8 ? &maps.k8 : &maps.k4;
+          const CUtensorMap* vmap = plane == 8 ? &maps.v8 : &maps.v4;
+          const int64_t krow_base = grp * (plane == 8 ? a.cap8 : static_cast<int64_t>(a.S));
+          const float* ks_base = (plane == 8 ? a.k8s : a.k4s) + grp * a.cap;
           if (elect_one()) {
-            bars->info[st] = make_int2(j, plane | (k_load == n_loads ? kLastLoad : 0));   // released by the arrive
+            bars->info[st] = make_int4(j0, j1, plane | (k_load == n_loads ? kLastLoad : 0), 0);   // released by the arrive
             mbar_arrive_expect_tx(&bars->kv_full[st], C::kStageTx);
-            tma_load_2d(sK(st), plane == 8 ? &maps.k8 : &maps.k4, &bars->kv_full[st], 0, krow);
+            if constexpr (C::kBlocksPerLoad == 1) {
+              // one block of 128 keys: K rows, two V sub-tiles of 64 keys, 128 scales
+              tma_load_2d(sK(st), kmap, &bars->kv_full[st], 0, static_cast<int>(krow_base + static_cast<int64_t>(j0) * T));
+              const int vrow = static_cast<int>((grp * a.nb + j0) * D);
+              tma_load_2d(sV(st), vmap, &bars->kv_full[st], 0, vrow);
+              tma_load_2d(sV(st) + C::kVSub, vmap, &bars->kv_full[st], 64, vrow);
+              bulk_load(sScale(st), ks_base + static_cast<int64_t>(j0) * T, kKeys * 4, &bars->kv_full[st]);
+            } else {
+              // two blocks of 64 keys (the second a copy of the first when alone)
+              const int jb[2] = {j0, j1 >= 0 ? j1 : j0};
 #pragma unroll
-            for (int q = 0; q < T / 64; ++q)
-              tma_load_2d(sV(st) + q * C::kVSub, plane == 8 ? &maps.v8 : &maps.v4, &bars->kv_full[st], 64 * q,
-                          vrow);
-            bulk_load(sScale(st), ks, T * 4, &bars->kv_full[st]);
+              for (int h = 0; h < 2; ++h) {
+                tma_load_2d(sK(st) + h * T * kQKRowBytes, kmap, &bars->kv_full[st], 0,
+                            static_cast<int>(krow_base + static_cast<int64_t>(jb[h]) * T));
+                tma_load_2d(sV(st) + h * C::kVSub, vmap, &bars->kv_full[st], 0, static_cast<int>((grp * a.nb + jb[h]) * D));
+                bulk_load(sScale(st) + h * T, ks_base + static_cast<int64_t>(jb[h]) * T, T * 4, &bars->kv_full[st]);
+              }
+            }
           }
           __syncwarp();
           ++g;
@@ -427,10 +488,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t vdesc = sw128_desc(vbase);
         if (elect_one()) {
 #pragma unroll
-          for (int s = 0; s < T / 16; ++s) {
+          for (int s = 0; s < kKeys / 16; ++s) {
             // +((s / 4) * sub-tile + (s % 4) * 32 bytes) in the descriptor's 16-byte units
             const uint64_t bdesc = vdesc + static_cast<uint64_t>(((s / 4) * C::kVSub + (s % 4) * 32) >> 4);
-            mma_bf16_ts(tmem + o_col(acc), tmem + sl * T + s * 8, bdesc, C::kIdescPV, (first && s == 0) ? 0u : 1u);
+            mma_bf16_ts(tmem + o_col(acc), tmem + sl * kKeys + s * 8, bdesc, C::kIdescPV, (first && s == 0) ? 0u : 1u);
           }
           mma_commit(&bars->kv_empty[st]);
         }
@@ -440,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (;; ++uloc) {
         const int r = uloc % kUnitRing;
         if (!(ok = warp_wait(&bars->unit_ready[r], (uloc / kUnitRing) & 1))) break;
-        if (bars->unit_w[r] < 0) break;                 // no more tiles
+        if (__shfl_sync(0xffffffffu, bars->unit_w[r], 0) < 0) break;   // no more tiles
         const int qb = uloc & 1;
         if (!(ok = warp_wait(&bars->q_full[qb], (uloc >> 1) & 1))) break;
         tc_fence_after();
@@ -457,9 +518,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         while (!last) {
           const int st = g % C::kStages, sl = g % C::kSlots;
           if (!(ok = warp_wait(&bars->kv_full[st], (g / C::kStages) & 1))) break;
-          const int2 inf = bars->info[st];
-          const int plane = inf.y & 0xff;
-          last = (inf.y & kLastLoad) != 0;
+          // broadcast through a shuffle and a vote, so that the compiler sees the
+          // loop, its counters and every operand derived from them as warp-uniform
+          const int4 inf = bars->info[st];
+          const int plane = __shfl_sync(0xffffffffu, inf.z & 0xff, 0);
+          last = __all_sync(0xffffffffu, (inf.z & kLastLoad) != 0);
           // the slot's previous S belonged to load g - kSlots: its P.V must be complete
           if (g >= static_cast<uint32_t>(C::kSlots)) {
             const uint32_t gp = g - C::kSlots;
@@ -472,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (elect_one()) {
 #pragma unroll
             for (int k = 0; k < kQKRowBytes / 32; ++k)   // +32 bytes along K = +2 descriptor units
-              mma_i8_ss(tmem + sl * T, adesc + 2 * k, bdesc + 2 * k, C::kIdescQK, k > 0 ? 1u : 0u);
+              mma_i8_ss(tmem + sl * kKeys, adesc + 2 * k, bdesc + 2 * k, C::kIdescQK, k > 0 ? 1u : 0u);
             mma_commit(&bars->s_full[sl]);
           }
           __syncwarp();
@@ -497,14 +560,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // ------------------------------------------------------------ softmax (warps 0-15)
-    constexpr int TH = T / 2;                 // keys of this thread per load
+    constexpr int TH = kKeys / 2;             // keys of this thread per load
     const int pair = warp / 8;                // load parity handled, S slot, O accumulator
     const int half = (warp / 4) % 2;          // which half of the keys
     const int sub = warp % 4;                 // TMEM lane quarter
     const int row = sub * 32 + lane;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(sub * 32) << 16);
-    const uint32_t my_s = lane_addr + half * TH;                     // + slot * T: S columns of my keys
-    const uint32_t my_p = lane_addr + half * (TH / 2);               // + slot * T: P words of my keys
+    const uint32_t my_s = lane_addr + half * TH;                     // + slot * kKeys: S columns of my keys
+    const uint32_t my_p = lane_addr + half * (TH / 2);               // + slot * kKeys: P words of my keys
     const uint32_t my_o = lane_addr + o_col(pair) + half * (D / 2);  // O columns rescaled here
     const uint32_t pair_bar = 1 + pair * 4 + sub;                    // 64 threads: this row's pair
     const uint32_t row_bar = 9 + sub;                                // 128 threads: all four of the row
@@ -535,39 +598,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t g0 = g, g_end = g0 + static_cast<uint32_t>(bars->unit_loads[r]);
       for (g = g0 + ((g0 % kPairs) == static_cast<uint32_t>(pair) ? 0u : 1u); g < g_end; g += kPairs) {
         const int st = g % C::kStages, sl = g % C::kSlots;
-        const uint32_t slot_col = static_cast<uint32_t>(sl * T);
+        const uint32_t slot_col = static_cast<uint32_t>(sl * kKeys);
         if (!(ok = mbar_wait(&bars->kv_full[st], (g / C::kStages) & 1, abort, a.err))) break;
         if (!(ok = mbar_wait(&bars->s_full[sl], (g / C::kSlots) & 1, abort, a.err))) break;
         tc_fence_after();
-        const int2 inf = bars->info[st];
-        const int j = inf.x, plane = inf.y & 0xff;
+        const int4 inf = bars->info[st];
+        const int plane = inf.z & 0xff;
+        // my keys: a half of the load's block at T = 128; at T = 64 the block of my
+        // half (j1 < 0: none, the half holds a masked copy)
+        const int jh = (C::kBlocksPerLoad == 1 || half == 0) ? inf.x : inf.y;
+        const int koff = C::kBlocksPerLoad == 1 ? half * TH : 0;   // my first key inside block jh
         const bool had_prev = g_mine >= 0;        // this pair's previous load (g - 2) is in this tile
         g_mine = g;
-        const int act = valid ? tile_action(ir, j, hi, keep) : ACT_NONE;   // uniform over the warp pair
-        if (act == plane) {
-          const int kmax = (j == ir) ? rl - half * TH : TH;   // my keys [0, kmax] are visible
+        // rows whose tile with block jh has another action (or none) write P = 0;
+        // uniform over the warp (its 32 rows are in one query block)
+        const int act = (valid && jh >= 0) ? tile_action(ir, jh, hi, keep) : ACT_NONE;
+        const bool active = act == plane;
+        const float alpha = plane == 8 ? a8 : a4;
+        const int kmax = (jh == ir) ? rl - koff : TH;   // my keys [0, kmax] are visible
+        float* xb = xmax + pair * 256;
+        // Both halves exchange their maxima on every load (an inactive half offers
+        // -inf) and take the same decision on the running maximum. Each half has
+        // read its S (tcgen05.wait::ld) before the barrier, so no P is stored over
+        // an S that the other half has yet to read.
+        float sc = 1.0f;
+        bool rescale_o = false;
+        auto exchange = [&](float m_half) {
+          xb[half * 128 + row] = m_half;
+          named_bar_sync(pair_bar, 64);
+          const float mt = fmaxf(m_half, xb[(1 - half) * 128 + row]);
+          const float m_tile = mt == -INFINITY ? -INFINITY : mt * alpha;
+          const bool raise = m_tile > m_run + kRescaleLog2;
+          sc = raise ? fast_exp2(m_run - m_tile) : 1.0f;
+          rescale_o = raise && m_run != -INFINITY;
+          if (raise) {
+            l_run *= sc;
+            m_run = m_tile;
+          }
+        };
+        if (active) {
           uint32_t r[TH];
 #pragma unroll
           for (int c = 0; c < TH / 32; ++c)
             tmem_ld32(my_s + slot_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
           const float* sk = sScale(st) + half * TH;
-          const float alpha = plane == 8 ? a8 : a4;
           tmem_wait_ld();
           uint64_t y[TH / 2];
           const bool masked = kmax < TH - 1;
-          const float m_half = masked ? scores_and_max<TH, true>(r, y, sk, kmax) : scores_and_max<TH, false>(r, y, sk, kmax);
-          // both halves have read their S (tcgen05.wait::ld above) before either stores P
-          float* xb = xmax + pair * 256;
-          xb[half * 128 + row] = m_half;
-          named_bar_sync(pair_bar, 64);
-          const float m_tile = fmaxf(m_half, xb[(1 - half) * 128 + row]) * alpha;
-          const bool raise = m_tile > m_run + kRescaleLog2;
-          const float sc = raise ? fast_exp2(m_run - m_tile) : 1.0f;
-          const bool rescale_o = raise && m_run != -INFINITY;
-          if (raise) {
-            l_run *= sc;
-            m_run = m_tile;
-          }
+          exchange(masked ? scores_and_max<TH, true>(r, y, sk, kmax) : scores_and_max<TH, false>(r, y, sk, kmax));
           const uint64_t al2 = pk2(alpha, alpha), nm2 = pk2(-m_run, -m_run);
           uint64_t acc[4] = {0, 0, 0, 0};
           {
@@ -579,6 +657,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           float s0, s1;
           up2(add2(add2(acc[0], acc[1]), add2(acc[2], acc[3])), s0, s1);
           l_run += s0 + s1;
+        } else {
+          exchange(-INFINITY);
+          uint32_t z[TH / 2];
+#pragma unroll
+          for (int k = 0; k < TH / 2; ++k) z[k] = 0u;
+          tmem_store_words<TH / 2>(my_p + slot_col, z);
+        }
+        {
           // Rescale this half's O columns when the maximum rose (before P.V of this load
           // may start). TMEM loads/stores are warp-collective: the whole warp takes part
           // when any lane must, lanes that need not using the factor 1.
@@ -604,11 +690,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               tmem_st32(my_o + 32 * c, o);
             }
           }
-        } else {
-          uint32_t z[TH / 2];
-#pragma unroll
-          for (int k = 0; k < TH / 2; ++k) z[k] = 0u;
-          tmem_store_words<TH / 2>(my_p + slot_col, z);
         }
         tmem_wait_st();
         tc_fence_before();
