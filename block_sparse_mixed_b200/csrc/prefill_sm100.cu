@@ -523,11 +523,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int4 inf = bars->info[st];
           const int plane = __shfl_sync(0xffffffffu, inf.z & 0xff, 0);
           last = __all_sync(0xffffffffu, (inf.z & kLastLoad) != 0);
-          // the slot's previous S belonged to load g - kSlots: its P.V must be complete
-          if (g >= static_cast<uint32_t>(C::kSlots)) {
-            const uint32_t gp = g - C::kSlots;
-            if (!(ok = warp_wait(&bars->kv_empty[gp % C::kStages], (gp / C::kStages) & 1))) break;
-          }
+          // The slot's previous S and P belonged to load g - kSlots, whose P.V was
+          // issued before this QK by this thread: tcgen05.mma operations of one
+          // thread execute in issue order, so that P.V has read P before this QK
+          // writes the slot, and no wait is needed here.
           tc_fence_after();
           const uint32_t abase = (plane == 8 ? q8a : q4a) + qoff;
           const uint32_t bbase = smem_u32(sK(st));
