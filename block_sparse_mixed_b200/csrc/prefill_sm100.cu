@@ -44,7 +44,7 @@ namespace {
 constexpr int kRows = 128;              // query rows per tile (tcgen05 M)
 constexpr int kThreads = 640;           // 20 warps
 constexpr int kSoftmaxWarps = 16;
-constexpr int kPairThreads = 256;       // softmax threads of one pair (P arrivals per load)
+constexpr int kPairWarps = 8;           // softmax warps of one pair (P arrivals per load, one per warp)
 constexpr int kProducerWarp = 16;
 constexpr int kMmaWarp = 17;
 // Register split (setmaxnreg): launched at 96 per thread (640 x 96 = 61,440; five
@@ -343,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int r = 0; r < kUnitRing; ++r) mbar_init(&bars->unit_ready[r], 1);
     for (int s = 0; s < C::kSlots; ++s) {
       mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->p_full[s], kPairThreads);
+      mbar_init(&bars->p_full[s], kPairWarps);
     }
     bars->abort = 0;
     fence_mbar_init();
@@ -690,9 +690,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
+        // every lane's P is in TMEM (wait::st) and ordered before the warp barrier
+        // (fence::before_thread_sync); one lane then arrives for the warp
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars->p_full[sl]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_full[sl]);
       }
       if (!ok) break;
       g = g_end;
