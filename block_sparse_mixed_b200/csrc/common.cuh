@@ -165,6 +165,27 @@ __device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+// D(tmem) (+)= A(smem desc) x B(smem desc), fp8 e4m3 x e4m3 -> fp32.
+__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// fp8 e4m3 byte of a 4-bit code c in [-7, 7]: exact (|c| = 2^e (1 + m/8) with a
+// 3-bit m), sign in bit 7. Codes outside the range are clamped.
+__host__ __device__ __forceinline__ uint32_t e4m3_of_code(int c) {
+  c = c < -7 ? -7 : (c > 7 ? 7 : c);
+  const int m = c < 0 ? -c : c;
+  // bytes of |c| = 0..7: 0x00 0x38 0x40 0x44 0x48 0x4A 0x4C 0x4E
+  const uint32_t b = static_cast<uint32_t>((0x4E4C4A4844403800ull >> (8 * m)) & 0xFFu);
+  return b | (c < 0 ? 0x80u : 0u);
+}
+
 // D(tmem) (+)= A(tmem) x B(smem desc), bf16 x bf16 -> fp32.
 __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                             uint32_t accumulate) {
@@ -258,6 +279,10 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
 __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
   return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
+}
+// kind::f8f6f4, e4m3 x e4m3 -> f32 (format code 0 for both operands), K-major, dense.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
+  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |

@@ -25,7 +25,7 @@ struct QuantArgs {
   int8_t* c8;
   int ld8;            // bytes per c8 row (D or 128; bytes past D are zeroed)
   uint8_t* c4p;       // packed 4-bit codes, D/2 bytes per row (optional)
-  int8_t* c4u;        // 4-bit codes one per byte (optional)
+  int8_t* c4u;        // 4-bit codes one fp8 e4m3 byte each (optional; the prefill QK operand)
   int ld4u;
   float* s8;
   float* s4;          // null: skip the 4-bit plane

@@ -93,7 +93,8 @@ struct Cfg {
   static constexpr int kSmemNeed = kOffX + kXBytes + 1024;
   static constexpr int kSmem = kSmemNeed > 120 * 1024 ? kSmemNeed : 120 * 1024;
   static constexpr uint32_t kStageTx = kKTile + kVTile + kKeys * 4;
-  static constexpr uint32_t kIdescQK = idesc_i8(kRows, kKeys);
+  static constexpr uint32_t kIdescQK = idesc_i8(kRows, kKeys);       // 8-bit plane: int8, int32 S
+  static constexpr uint32_t kIdescQK4 = idesc_e4m3(kRows, kKeys);    // 4-bit plane: e4m3, fp32 S (exact)
   static constexpr uint32_t kIdescPV = idesc_bf16(kRows, D);
 };
 
@@ -259,16 +260,17 @@ __device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
 
 // Softmax pass 1 over N keys of a row: y = float(acc) * s_k as packed pairs, and
 // the maximum over the visible keys (n <= kmax when MASK).
-template <int N, bool MASK>
+// FP: S holds fp32 (the 4-bit plane's e4m3 product, an exact integer) instead of int32.
+template <int N, bool MASK, bool FP>
 __device__ __forceinline__ float scores_and_max(const uint32_t (&r)[N], uint64_t (&y)[N / 2], const float* sk,
                                                 int kmax) {
+  auto cv = [](uint32_t v) { return FP ? __uint_as_float(v) : __int2float_rn(static_cast<int>(v)); };
   float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
   for (int q = 0; q < N / 4; ++q) {
     const float4 s4 = *reinterpret_cast<const float4*>(sk + 4 * q);
-    const uint64_t u01 = pk2(__int2float_rn(static_cast<int>(r[4 * q])), __int2float_rn(static_cast<int>(r[4 * q + 1])));
-    const uint64_t u23 =
-        pk2(__int2float_rn(static_cast<int>(r[4 * q + 2])), __int2float_rn(static_cast<int>(r[4 * q + 3])));
+    const uint64_t u01 = pk2(cv(r[4 * q]), cv(r[4 * q + 1]));
+    const uint64_t u23 = pk2(cv(r[4 * q + 2]), cv(r[4 * q + 3]));
     y[2 * q] = mul2(u01, pk2(s4.x, s4.y));
     y[2 * q + 1] = mul2(u23, pk2(s4.z, s4.w));
     float v0, v1, v2, v3;
@@ -534,7 +536,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (elect_one()) {
 #pragma unroll
             for (int k = 0; k < kQKRowBytes / 32; ++k)   // +32 bytes along K = +2 descriptor units
-              mma_i8_ss(tmem + sl * kKeys, adesc + 2 * k, bdesc + 2 * k, C::kIdescQK, k > 0 ? 1u : 0u);
+              if (plane == 8)
+                mma_i8_ss(tmem + sl * kKeys, adesc + 2 * k, bdesc + 2 * k, C::kIdescQK, k > 0 ? 1u : 0u);
+              else
+                mma_f8_ss(tmem + sl * kKeys, adesc + 2 * k, bdesc + 2 * k, C::kIdescQK4, k > 0 ? 1u : 0u);
             mma_commit(&bars->s_full[sl]);
           }
           __syncwarp();
@@ -644,7 +649,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
           uint64_t y[TH / 2];
           const bool masked = kmax < TH - 1;
-          exchange(masked ? scores_and_max<TH, true>(r, y, sk, kmax) : scores_and_max<TH, false>(r, y, sk, kmax));
+          float mh;
+          if (plane == 8) mh = masked ? scores_and_max<TH, true, false>(r, y, sk, kmax) : scores_and_max<TH, false, false>(r, y, sk, kmax);
+          else mh = masked ? scores_and_max<TH, true, true>(r, y, sk, kmax) : scores_and_max<TH, false, true>(r, y, sk, kmax);
+          exchange(mh);
           const uint64_t al2 = pk2(alpha, alpha), nm2 = pk2(-m_run, -m_run);
           uint64_t acc[4] = {0, 0, 0, 0};
           {
