@@ -8,21 +8,30 @@
 // diagonal always 8-bit, far blocks skipped), reduced into one normalised
 // output O and its natural log-sum-exp.
 //
-// How. A persistent CTA owns one 128-row query tile at a time (one query block
-// of T = 128, or two query blocks of T = 64) of one (batch, query head). The
-// key blocks the tile keeps are walked in ascending order; a key block whose
-// rows need both planes is loaded once per plane ("load" below = one kept
-// (key block, plane) pair). Warp roles:
+// How. A persistent CTA takes 128-row query tiles (one query block of T = 128,
+// or two query blocks of T = 64, of one (batch, query head)) from a kernel-wide
+// counter, longest rows first. A tile's kept (key block, plane) pairs are walked
+// in ascending order by the producer only, and grouped into loads of 128 keys:
+// one block at T = 128, two blocks of the same plane at T = 64 (a block whose
+// neighbour has the other plane goes alone, its copy in the second half masked).
+// Warp roles:
 //   warps 0-15  softmax, as two "pairs" of warpgroups that take the loads in
 //               turn (ping-pong: pair p handles loads of parity p, using S slot p
 //               and O accumulator p in TMEM). Inside a pair, warpgroup `half`
-//               takes keys [half*T/2, (half+1)*T/2) of every row; the two halves
-//               of a row agree on its maximum through shared memory and a named
-//               barrier. Four softmax warps per SM sub-partition hide latency.
-//   warp 16     producer: TMA loads of Q codes, K codes, V tiles and K scales,
-//               only for kept (block, plane) pairs;
-//   warp 17     MMA issuer: S = Q.K^T on tcgen05 kind::i8 (int32 in TMEM), then
-//               O += P.V on tcgen05 kind::f16 (bf16 P read from TMEM, fp32 O in TMEM).
+//               takes keys [64 half, 64 half + 64) of every row (its own key block
+//               at T = 64); the two halves agree on the row maximum through shared
+//               memory and a named barrier.
+//   warp 16     producer: tile index and load count (a ring of 8 entries), the
+//               tile's Q codes into one of two buffers, then per load the key
+//               blocks, plane and last-of-tile flag with the K codes, V tiles and
+//               K scales (TMA, no multicast), only for kept blocks;
+//   warp 17     MMA issuer: S = Q.K^T on tcgen05 (kind::i8 with int32 S for the
+//               8-bit plane; kind::f8f6f4 on e4m3 operands, exact for 4-bit codes,
+//               with fp32 S for the 4-bit plane), then O += P.V on kind::f16 (bf16
+//               P read from TMEM, fp32 O in TMEM). QK of a load is issued before
+//               the P.V of the load before it; tcgen05.mma operations of one thread
+//               run in issue order, which also keeps a slot's P alive until its
+//               P.V has read it.
 //   warps 18-19 only take part in the register hand-over.
 // The softmax dequantises S with the row's Q scale and the key's K scale,
 // masks the diagonal block causally, keeps a running maximum that is only
