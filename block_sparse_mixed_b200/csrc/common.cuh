@@ -93,6 +93,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// As mbar_wait, but gives up only at its own limit, not on another role's abort:
+// threads that must leave a loop at the same point (partners in a named barrier)
+// wait on the same phases, and a phase that never completes fails all of them,
+// while the abort flag could be seen by one and not by the other.
+__device__ __forceinline__ bool mbar_wait_shared(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                 int* err) {
+  constexpr uint32_t kSleepNs = 1000000;  // 1 ms
+  if (mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
+  const unsigned long long t0 = global_timer();
+  while (true) {
+    if (mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
+    if (global_timer() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      atomicExch(err, TRIA_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // One lane of the (converged) warp returns true. Loops that issue TMA copies or
 // tensor-core ops run on the whole warp so their operands stay warp-uniform
 // (uniform registers); only the elected lane issues.
@@ -195,6 +214,23 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// D(tmem) (+)= A(smem desc) x B(smem desc), bf16 x bf16 -> fp32.
+__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (tensor-core operand reads, TMA) once a later synchronisation orders them.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // Arrive on `bar` once every tcgen05.mma issued so far by this thread completes.

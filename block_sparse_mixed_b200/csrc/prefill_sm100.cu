@@ -11,34 +11,37 @@
 // How. A persistent CTA takes 128-row query tiles (one query block of T = 128,
 // or two query blocks of T = 64, of one (batch, query head)) from a kernel-wide
 // counter, longest rows first. A tile's kept (key block, plane) pairs are walked
-// in ascending order by the producer only, and grouped into loads of 128 keys:
-// one block at T = 128, two blocks of the same plane at T = 64 (a block whose
-// neighbour has the other plane goes alone, its copy in the second half masked).
-// Warp roles:
+// by the producers only: first the 8-bit blocks, then the 4-bit ones, grouped into
+// loads of 128 keys (one block at T = 128; any two blocks of one plane at T = 64,
+// a lone block's copy in the second half masked). Warp roles:
 //   warps 0-15  softmax, as two "pairs" of warpgroups that take the loads in
-//               turn (ping-pong: pair p handles loads of parity p, using S slot p
-//               and O accumulator p in TMEM). Inside a pair, warpgroup `half`
-//               takes keys [64 half, 64 half + 64) of every row (its own key block
-//               at T = 64); the two halves agree on the row maximum through shared
-//               memory and a named barrier.
-//   warp 16     producer: tile index and load count (a ring of 8 entries), the
-//               tile's Q codes into one of two buffers, then per load the key
-//               blocks, plane and last-of-tile flag with the K codes, V tiles and
-//               K scales (TMA, no multicast), only for kept blocks;
-//   warp 17     MMA issuer: S = Q.K^T on tcgen05 (kind::i8 with int32 S for the
+//               turn (pair p handles loads of parity p, with S slot p in TMEM, P
+//               buffer p in shared memory and O accumulator p in TMEM). Inside a
+//               pair, warpgroup `half` takes keys [64 half, 64 half + 64) of every
+//               row (its own key block at T = 64); the two halves agree on the row
+//               maximum through shared memory and a named barrier.
+//   warp 16     producer: tile index and load count (a ring of 16 entries), the
+//               tile's Q codes, then per load the K codes (a ring of 3 stages) and
+//               the K scales with the load's blocks, plane and last-of-tile flag (a
+//               ring of 4 stages). TMA, no multicast, only kept blocks.
+//   warp 17     QK issuer: S = Q.K^T on tcgen05 (kind::i8 with int32 S for the
 //               8-bit plane; kind::f8f6f4 on e4m3 operands, exact for 4-bit codes,
-//               with fp32 S for the 4-bit plane), then O += P.V on kind::f16 (bf16
-//               P read from TMEM, fp32 O in TMEM). QK of a load is issued before
-//               the P.V of the load before it; tcgen05.mma operations of one thread
-//               run in issue order, which also keeps a slot's P alive until its
-//               P.V has read it.
-//   warps 18-19 only take part in the register hand-over.
-// The softmax dequantises S with the row's Q scale and the key's K scale,
-// masks the diagonal block causally, keeps a running maximum that is only
-// raised when it grows by more than 2^8 (so O is rarely rescaled), and writes P
-// as bf16 over the S columns. Rows whose own tile action differs from the
-// load's plane write P = 0. The two accumulators of a row are merged and
-// normalised in the tile epilogue.
+//               with fp32 S for the 4-bit plane). A pair's slot is refilled as soon
+//               as the pair has read S into registers, so the next S of a pair is
+//               computed while the pair still works on the current one.
+//   warp 18     producer of the V tiles (a ring of 2 stages, one per pair).
+//   warp 19     P.V issuer: O += P.V on kind::f16, bf16 P and V from shared memory,
+//               fp32 O in TMEM; each P.V frees its V stage, P buffer and the
+//               accumulator for the pair's next load.
+// Each ring is released as soon as its contents are used (K by the QK's
+// completion, the scales after the softmax's first pass, V and P by the P.V's
+// completion), so no stage is held across another role's round trip.
+// The softmax dequantises S with the row's Q scale and the key's K scale, masks
+// the diagonal block causally, keeps a running maximum that is only raised when
+// it grows by more than 2^8 (so O is rarely rescaled), and writes P as bf16 into
+// the pair's buffer in the swizzled K-major layout the tensor core reads. Rows
+// whose own tile action differs from the load's plane write P = 0. The two
+// accumulators of a row are merged and normalised in the tile epilogue.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -54,8 +57,10 @@ constexpr int kRows = 128;              // query rows per tile (tcgen05 M)
 constexpr int kThreads = 640;           // 20 warps
 constexpr int kSoftmaxWarps = 16;
 constexpr int kPairWarps = 8;           // softmax warps of one pair (P arrivals per load, one per warp)
-constexpr int kProducerWarp = 16;
-constexpr int kMmaWarp = 17;
+constexpr int kProducerWarp = 16;       // Q, K codes, K scales
+constexpr int kMmaWarp = 17;            // QK issuer; allocates TMEM
+constexpr int kVProducerWarp = 18;      // V tiles
+constexpr int kPvWarp = 19;             // P.V issuer
 // Register split (setmaxnreg): launched at 96 per thread (640 x 96 = 61,440; five
 // warps per sub-partition x 32 x 96 = 15,360 of its 16,384); the four softmax
 // warpgroups rise to 104 and the producer/MMA warpgroup drops to 64:
@@ -78,86 +83,100 @@ template <int T, int D>
 struct Cfg {
   static constexpr int kQBlocks = kRows / T;                 // query blocks per tile
   static constexpr int kBlocksPerLoad = kKeys / T;           // key blocks per load
-  static constexpr int kKTile = kKeys * kQKRowBytes;         // K codes per stage
+  static constexpr int kQTile = kRows * kQKRowBytes;         // Q codes of one plane
+  static constexpr int kKTile = kKeys * kQKRowBytes;         // K codes of one load
   static constexpr int kVSub = D * 128;                      // one V sub-tile: D rows x 64 keys
-  static constexpr int kVTile = D * kKeys * 2;               // all V sub-tiles of a stage
-  static constexpr int kStageRaw = kKTile + kVTile + kKeys * 4;   // + K scales
-  static constexpr int kStage = (kStageRaw + 1023) / 1024 * 1024;
-  static constexpr int kStages = 3;
-  // S buffers in TMEM (kKeys columns each, below the O accumulators at 256); QK
-  // of a load is issued before the P.V of the load before it.
-  static constexpr int kSlots = 2;
-  static constexpr int kLead = kSlots / 2;
-  static constexpr int kQTile = kRows * kQKRowBytes;
-  // Q codes of two tiles (both planes each): the next tile's Q is loaded while
-  // the current one is in use
-  static constexpr int kOffQ8 = 0;                           // + buffer * 2 * kQTile
+  static constexpr int kVTile = D * kKeys * 2;               // both V sub-tiles of a load
+  static constexpr int kPSub = kRows * 128;                  // one P sub-tile: 128 rows x 64 keys
+  static constexpr int kPTile = kRows * kKeys * 2;           // P of one load (bf16)
+  static constexpr int kScTile = kKeys * 4;                  // K scales of one load
+  // Rings. K codes are released when the QK that reads them completes, V when
+  // its P.V completes, and the K scales when the softmax has read them, so each
+  // kind of operand is held only as long as it is used.
+  static constexpr int kKStages = 3;
+  static constexpr int kVStages = 2;                         // = pairs: stage g % 2 is pair g % 2's
+  static constexpr int kScStages = 4;
+  static constexpr int kSlots = 2;                           // S slots in TMEM, one per pair
+  static constexpr int kOffQ8 = 0;
   static constexpr int kOffQ4 = kQTile;
-  static constexpr int kOffStage = 4 * kQTile;
-  static constexpr int kOffBar = kOffStage + kStages * kStage;
+  static constexpr int kOffK = 2 * kQTile;
+  static constexpr int kOffV = kOffK + kKStages * kKTile;
+  static constexpr int kOffP = kOffV + kVStages * kVTile;    // P buffer of pair p at kOffP + p * kPTile
+  static constexpr int kOffSc = kOffP + 2 * kPTile;
+  static constexpr int kOffBar = kOffSc + kScStages * kScTile;
   static constexpr int kOffX = kOffBar + 1024;               // row-max and epilogue exchanges
   static constexpr int kXBytes = 2 * 2 * 128 * 4 + 2 * 2 * 2 * 2 * 128 * 4;   // 2 KB + 8 KB
   // never below 120 KB so that exactly one CTA (which owns all 512 TMEM columns)
   // is resident per SM
   static constexpr int kSmemNeed = kOffX + kXBytes + 1024;
   static constexpr int kSmem = kSmemNeed > 120 * 1024 ? kSmemNeed : 120 * 1024;
-  static constexpr uint32_t kStageTx = kKTile + kVTile + kKeys * 4;
+  static_assert(kSmemNeed <= 227 * 1024, "shared memory");
+  static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0 && kKTile % 1024 == 0 &&
+                    kVSub % 1024 == 0 && kPSub % 1024 == 0,
+                "swizzled operand tiles start on 1024-byte boundaries");
   static constexpr uint32_t kIdescQK = idesc_i8(kRows, kKeys);       // 8-bit plane: int8, int32 S
   static constexpr uint32_t kIdescQK4 = idesc_e4m3(kRows, kKeys);    // 4-bit plane: e4m3, fp32 S (exact)
   static constexpr uint32_t kIdescPV = idesc_bf16(kRows, D);
 };
 
-constexpr int kUnitRing = 8;            // tiles published ahead of the consumers
+constexpr int kUnitRing = 16;           // tiles published ahead of the consumers
 
 struct Bars {
-  uint64_t q_full[2], q_empty[2], fin;  // Q buffer b holds the CTA's tiles u with u % 2 == b
+  uint64_t q_full, q_empty, fin, fin_pv;
   uint64_t o_fin;               // every P.V of the CTA's u-th tile: phase u
-  // kv_empty[st] completes when the P.V of the load in stage st completes: it also
-  // tells the MMA warp that the S slot of that load is free, and the softmax that
-  // the O accumulator it wrote may be rescaled
-  uint64_t kv_full[6], kv_empty[6];
-  uint64_t s_full[4], p_full[4];
+  uint64_t k_full[3], k_empty[3];       // K ring: emptied by the QK's completion
+  uint64_t v_full[2], v_empty[2];       // V ring: emptied by the P.V's completion, which
+                                        // also frees the pair's P buffer and O accumulator
+  uint64_t sc_full[4], sc_empty[4];     // K scales + load info: emptied by the softmax pair
+  uint64_t s_full[2], s_free[2];        // S slot written by QK / read out by the pair
+  uint64_t p_full[2];                   // the pair's P buffer written
+
   uint32_t tmem_base;
   int abort;
-  // Published by the producer so that no other role walks the load sequence:
-  // per stage, the load's key block and plane (kLastLoad marks a tile's last
-  // load), visible after kv_full; per tile u of this CTA, the tile's index and
-  // load count in ring entry u % kUnitRing (index -1: no more tiles), visible
-  // after phase u / kUnitRing of unit_ready[u % kUnitRing]. The ring cannot be
-  // lapped: a tile has at least one load, and the producer runs at most kStages
-  // loads ahead of the P.V that needs the slowest softmax pair.
-  int4 info[6];                 // (j0, j1, plane | kLastLoad, 0)
+  // Published by the producer so that the other roles need not walk the load
+  // sequence: per K stage and per scale stage the load's key blocks and plane
+  // (kLastLoad marks a tile's last load), visible after the stage's full barrier;
+  // per tile u of this CTA, the tile's index and load count in ring entry
+  // u % kUnitRing (index -1: no more tiles), visible after phase u / kUnitRing of
+  // unit_ready[u % kUnitRing]. The ring cannot be lapped: a tile has at least one
+  // load, and the producer runs at most a few loads ahead of the slowest reader.
+  int4 k_info[3], sc_info[4];   // (j0, j1, plane | kLastLoad, 0)
   int unit_w[kUnitRing], unit_loads[kUnitRing];
   uint64_t unit_ready[kUnitRing];
 };
+static_assert(sizeof(Bars) <= 1024, "barrier block");
 
-// The (key block, plane) loads of one query tile, in ascending key-block order;
-// at a key block the 8-bit load (if any row needs it) comes before the 4-bit one.
+// The (key block, plane) loads of one query tile: first every block that some row
+// of the tile reads at 8 bits (block 0, then ascending from the band), then every
+// block read at 4 bits, ascending. Grouping by plane lets the pairing below join
+// any two blocks of one plane, so a tile has at most one lone block per plane. The
+// order of a row's key blocks does not change its softmax (the running maximum
+// and sum are merged exactly up to rounding).
 struct LoadSeq {
-  int i0, nq, hi, keep, j, jmax, jband, step;
+  int i0, nq, hi, keep, j, jmax, jband, j8, plane;
   __device__ void init(int i0_, int nq_, int hi_, int keep_) {
     i0 = i0_; nq = nq_; hi = hi_; keep = keep_;
-    jmax = i0 + nq - 1; j = 0; step = 0;
+    jmax = i0 + nq - 1; j = 0; plane = 8;
     jband = first_band_block(i0, keep);
+    // 8-bit blocks after block 0: d < hi or the diagonal, so none before i0 - hi + 1
+    const int lo = i0 - hi + 1 < i0 ? i0 - hi + 1 : i0;
+    j8 = lo > jband ? lo : jband;
   }
-  __device__ bool next(int& jo, int& plane) {
-    while (j <= jmax) {
-      bool n8 = false, n4 = false;
-      for (int q = 0; q < nq; ++q) {
-        const int a = tile_action(i0 + q, j, hi, keep);
-        n8 |= a == ACT_INT8;
-        n4 |= a == ACT_INT4;
+  __device__ bool next(int& jo, int& plane_out) {
+    while (true) {
+      if (j > jmax) {
+        if (plane == 4) return false;
+        plane = 4;                       // second pass: the 4-bit blocks of the band
+        j = jband;
+        continue;
       }
-      if (step == 0) {
-        step = 1;
-        if (n8) { jo = j; plane = 8; return true; }
-      }
-      step = 0;
+      const int want = plane == 8 ? ACT_INT8 : ACT_INT4;
+      bool need = false;
+      for (int q = 0; q < nq; ++q) need |= tile_action(i0 + q, j, hi, keep) == want;
       const int jj = j;
-      j = (j == 0) ? jband : j + 1;
-      if (n4) { jo = jj; plane = 4; return true; }
+      j = (plane == 8 && j == 0) ? j8 : j + 1;
+      if (need) { jo = jj; plane_out = plane; return true; }
     }
-    return false;
   }
 };
 
@@ -165,8 +184,8 @@ constexpr int kLastLoad = 1 << 8;       // flag in info[].z next to the plane
 
 // The 128-key loads of a tile: with one key block per load (T = 128) the
 // (block, plane) pairs of LoadSeq, each as (j, j); with two (T = 64) consecutive
-// pairs of the same plane merged into (j0, j1), and a block whose neighbour in
-// the sequence has the other plane alone as (j0, -1).
+// blocks of one plane merged into (j0, j1), and the last block of a plane's odd
+// count alone as (j0, -1).
 template <int BPL>
 struct LoadPairs {
   LoadSeq seq;
@@ -298,32 +317,29 @@ __device__ __forceinline__ float scores_and_max(const uint32_t (&r)[N], uint64_t
   return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
 }
 
-// Softmax pass 2 over N keys: p = 2^(y * alpha - m) packed to bf16 pairs, their
+// Softmax pass 2 over N keys: p = 2^(y * alpha - m) as bf16 pairs, stored as they
+// are made into the thread's 128-byte P row (16-byte chunk c at c ^ swz), their
 // fp32 sum accumulated in `acc`; masked keys (n > kmax when MASK) give 0.
 template <int N, bool MASK>
 __device__ __forceinline__ void probs(const uint64_t (&y)[N / 2], uint64_t al2, uint64_t nm2, int kmax,
-                                      uint32_t (&pk)[N / 2], uint64_t (&acc)[4]) {
+                                      uint8_t* prow, int swz, uint64_t (&acc)[4]) {
 #pragma unroll
-  for (int k = 0; k < N / 2; ++k) {
-    float t0, t1;
-    up2(fma2(y[k], al2, nm2), t0, t1);
-    float e0 = fast_exp2(t0), e1 = fast_exp2(t1);
-    if (MASK) {
-      e0 = 2 * k <= kmax ? e0 : 0.0f;
-      e1 = 2 * k + 1 <= kmax ? e1 : 0.0f;
+  for (int c = 0; c < N / 8; ++c) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int k = 4 * c + e;
+      float t0, t1;
+      up2(fma2(y[k], al2, nm2), t0, t1);
+      float e0 = fast_exp2(t0), e1 = fast_exp2(t1);
+      if (MASK) {
+        e0 = 2 * k <= kmax ? e0 : 0.0f;
+        e1 = 2 * k + 1 <= kmax ? e1 : 0.0f;
+      }
+      acc[k % 4] = add2(acc[k % 4], pk2(e0, e1));
+      w[e] = bf16x2(e0, e1);
     }
-    acc[k % 4] = add2(acc[k % 4], pk2(e0, e1));
-    pk[k] = bf16x2(e0, e1);
-  }
-}
-
-template <int N>
-__device__ __forceinline__ void tmem_store_words(uint32_t taddr, const uint32_t (&w)[N]) {
-  static_assert(N == 16 || N == 32, "P stores are 16 or 32 columns");
-  if constexpr (N == 32) {
-    tmem_st32(taddr, w);
-  } else {
-    tmem_st16(taddr, w);
+    *reinterpret_cast<uint4*>(prow + ((c ^ swz) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
@@ -341,19 +357,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x % 32;
 
   if (threadIdx.x == 0) {
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars->q_full[b], 1);
-      mbar_init(&bars->q_empty[b], 1);
-    }
+    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 1);
     mbar_init(&bars->fin, 1);
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&bars->kv_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);
-    }
+    mbar_init(&bars->fin_pv, 1);
     mbar_init(&bars->o_fin, 1);
+    for (int s = 0; s < C::kKStages; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < C::kVStages; ++s) {
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
+    }
+    for (int s = 0; s < C::kScStages; ++s) {
+      mbar_init(&bars->sc_full[s], 1);
+      mbar_init(&bars->sc_empty[s], kPairWarps);
+    }
     for (int r = 0; r < kUnitRing; ++r) mbar_init(&bars->unit_ready[r], 1);
     for (int s = 0; s < C::kSlots; ++s) {
       mbar_init(&bars->s_full[s], 1);
+      mbar_init(&bars->s_free[s], kPairWarps);
       mbar_init(&bars->p_full[s], kPairWarps);
     }
     bars->abort = 0;
@@ -366,6 +390,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kProducerWarp && lane == 0) {
     prefetch_tensormap(&maps.q8); prefetch_tensormap(&maps.q4);
     prefetch_tensormap(&maps.k8); prefetch_tensormap(&maps.k4);
+  }
+  if (warp == kVProducerWarp && lane == 0) {
     prefetch_tensormap(&maps.v8); prefetch_tensormap(&maps.v4);
   }
   tc_fence_before();
@@ -388,11 +414,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint8_t* sQ8 = smem + C::kOffQ8;
   uint8_t* sQ4 = smem + C::kOffQ4;
-  auto sK = [&](int s) { return smem + C::kOffStage + s * C::kStage; };
-  auto sV = [&](int s) { return smem + C::kOffStage + s * C::kStage + C::kKTile; };
-  auto sScale = [&](int s) {
-    return reinterpret_cast<float*>(smem + C::kOffStage + s * C::kStage + C::kKTile + C::kVTile);
-  };
+  auto sK = [&](int s) { return smem + C::kOffK + s * C::kKTile; };
+  auto sV = [&](int s) { return smem + C::kOffV + s * C::kVTile; };
+  auto sP = [&](int p) { return smem + C::kOffP + p * C::kPTile; };
+  auto sScale = [&](int s) { return reinterpret_cast<float*>(smem + C::kOffSc + s * C::kScTile); };
 
   if (warp >= kSoftmaxWarps) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
@@ -403,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, a.err));
     };
     if (warp == kProducerWarp) {
-      // ---------------------------------------------------------- producer
+      // ---------------------------------------------------------- producer: Q, K, scales
       uint32_t g = 0, uloc = 0;
       bool ok = true;
       for (;; ++uloc) {
@@ -428,17 +453,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           int j0, j1, pp;
           while (cnt.next(j0, j1, pp)) ++n_loads;
         }
-        // Q buffer uloc % 2 is free once the QKs of this CTA's tile uloc - 2 are done
-        const int qb = uloc & 1;
-        if (uloc >= 2 && !(ok = warp_wait(&bars->q_empty[qb], ((uloc >> 1) - 1) & 1))) break;
-        const int qrow = (u.b * a.Hq + u.hq) * a.S + u.i0 * T;
         if (elect_one()) {
           bars->unit_w[r] = w;
           bars->unit_loads[r] = n_loads;
           mbar_arrive(&bars->unit_ready[r]);   // release: the entry is visible after the wait
-          mbar_arrive_expect_tx(&bars->q_full[qb], 2 * C::kQTile);
-          tma_load_2d(sQ8 + qb * 2 * C::kQTile, &maps.q8, &bars->q_full[qb], 0, qrow);
-          tma_load_2d(sQ4 + qb * 2 * C::kQTile, &maps.q4, &bars->q_full[qb], 0, qrow);
+        }
+        __syncwarp();
+        // the Q buffer is free once the last QK of the previous tile has completed
+        if (uloc >= 1 && !(ok = warp_wait(&bars->q_empty, (uloc - 1) & 1))) break;
+        const int qrow = (u.b * a.Hq + u.hq) * a.S + u.i0 * T;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(&bars->q_full, 2 * C::kQTile);
+          tma_load_2d(sQ8, &maps.q8, &bars->q_full, 0, qrow);
+          tma_load_2d(sQ4, &maps.q4, &bars->q_full, 0, qrow);
         }
         __syncwarp();
         LoadPairs<C::kBlocksPerLoad> seq;
@@ -446,34 +473,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t grp = static_cast<int64_t>(u.b) * a.Hkv + u.kvh;
         int j0, j1, plane, k_load = 0;
         while (seq.next(j0, j1, plane)) {
-          const int st = g % C::kStages;
-          if (g >= static_cast<uint32_t>(C::kStages) && !(ok = warp_wait(&bars->kv_empty[st], ((g / C::kStages) - 1) & 1)))
+          const int ks = g % C::kKStages, ss = g % C::kScStages;
+          if (g >= static_cast<uint32_t>(C::kKStages) &&
+              !(ok = warp_wait(&bars->k_empty[ks], ((g / C::kKStages) - 1) & 1)))
+            break;
+          if (g >= static_cast<uint32_t>(C::kScStages) &&
+              !(ok = warp_wait(&bars->sc_empty[ss], ((g / C::kScStages) - 1) & 1)))
             break;
           ++k_load;
           const CUtensorMap* kmap = plane == 8 ? &maps.k8 : &maps.k4;
-          const CUtensorMap* vmap = plane == 8 ? &maps.v8 : &maps.v4;
           const int64_t krow_base = grp * (plane == 8 ? a.cap8 : static_cast<int64_t>(a.S));
           const float* ks_base = (plane == 8 ? a.k8s : a.k4s) + grp * a.cap;
           if (elect_one()) {
-            bars->info[st] = make_int4(j0, j1, plane | (k_load == n_loads ? kLastLoad : 0), 0);   // released by the arrive
-            mbar_arrive_expect_tx(&bars->kv_full[st], C::kStageTx);
-            if constexpr (C::kBlocksPerLoad == 1) {
-              // one block of 128 keys: K rows, two V sub-tiles of 64 keys, 128 scales
-              tma_load_2d(sK(st), kmap, &bars->kv_full[st], 0, static_cast<int>(krow_base + static_cast<int64_t>(j0) * T));
-              const int vrow = static_cast<int>((grp * a.nb + j0) * D);
-              tma_load_2d(sV(st), vmap, &bars->kv_full[st], 0, vrow);
-              tma_load_2d(sV(st) + C::kVSub, vmap, &bars->kv_full[st], 64, vrow);
-              bulk_load(sScale(st), ks_base + static_cast<int64_t>(j0) * T, kKeys * 4, &bars->kv_full[st]);
-            } else {
-              // two blocks of 64 keys (the second a copy of the first when alone)
-              const int jb[2] = {j0, j1 >= 0 ? j1 : j0};
+            const int4 inf = make_int4(j0, j1, plane | (k_load == n_loads ? kLastLoad : 0), 0);
+            bars->k_info[ks] = inf;    // released by the arrives below
+            bars->sc_info[ss] = inf;
+            mbar_arrive_expect_tx(&bars->k_full[ks], C::kKTile);
+            mbar_arrive_expect_tx(&bars->sc_full[ss], C::kScTile);
+            // 128 keys: one block at T = 128; two blocks of 64 at T = 64 (the second a
+            // copy of the first when alone)
+            const int jb[2] = {j0, (C::kBlocksPerLoad == 1 || j1 < 0) ? j0 : j1};
 #pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                tma_load_2d(sK(st) + h * T * kQKRowBytes, kmap, &bars->kv_full[st], 0,
-                            static_cast<int>(krow_base + static_cast<int64_t>(jb[h]) * T));
-                tma_load_2d(sV(st) + h * C::kVSub, vmap, &bars->kv_full[st], 0, static_cast<int>((grp * a.nb + jb[h]) * D));
-                bulk_load(sScale(st) + h * T, ks_base + static_cast<int64_t>(jb[h]) * T, T * 4, &bars->kv_full[st]);
-              }
+            for (int h = 0; h < C::kBlocksPerLoad; ++h) {
+              tma_load_2d(sK(ks) + h * T * kQKRowBytes, kmap, &bars->k_full[ks], 0,
+                          static_cast<int>(krow_base + static_cast<int64_t>(jb[h]) * T));
+              bulk_load(sScale(ss) + h * T, ks_base + static_cast<int64_t>(jb[h]) * T, T * 4, &bars->sc_full[ss]);
             }
           }
           __syncwarp();
@@ -482,66 +506,83 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
       }
       // let every copy this CTA issued land before the block exits
-      for (uint32_t k = (g > static_cast<uint32_t>(C::kStages) ? g - C::kStages : 0); k < g; ++k)
-        drain_wait(&bars->kv_full[k % C::kStages], (k / C::kStages) & 1);
-      for (uint32_t k = (uloc > 2 ? uloc - 2 : 0); k < uloc; ++k) drain_wait(&bars->q_full[k & 1], (k >> 1) & 1);
+      for (uint32_t k = (g > static_cast<uint32_t>(C::kKStages) ? g - C::kKStages : 0); k < g; ++k)
+        drain_wait(&bars->k_full[k % C::kKStages], (k / C::kKStages) & 1);
+      for (uint32_t k = (g > static_cast<uint32_t>(C::kScStages) ? g - C::kScStages : 0); k < g; ++k)
+        drain_wait(&bars->sc_full[k % C::kScStages], (k / C::kScStages) & 1);
+      if (uloc >= 1) drain_wait(&bars->q_full, (uloc - 1) & 1);
+    } else if (warp == kVProducerWarp) {
+      // ---------------------------------------------------------- producer: V
+      // Walks the same tiles (from the ring) and loads; a V stage is refilled only
+      // when the P.V that read it has completed, which never holds up K or Q.
+      uint32_t g = 0, uloc = 0;
+      bool ok = true;
+      for (;; ++uloc) {
+        const int r = uloc % kUnitRing;
+        if (!(ok = warp_wait(&bars->unit_ready[r], (uloc / kUnitRing) & 1))) break;
+        const int w = __shfl_sync(0xffffffffu, bars->unit_w[r], 0);
+        if (w < 0) break;
+        const Unit u = unit_of(a, w, C::kQBlocks);
+        LoadPairs<C::kBlocksPerLoad> seq;
+        seq.init(u.i0, u.nq, a.hi[u.hq], a.keep[u.hq]);
+        const int64_t grp = static_cast<int64_t>(u.b) * a.Hkv + u.kvh;
+        int j0, j1, plane;
+        while (seq.next(j0, j1, plane)) {
+          const int vs = g % C::kVStages;
+          if (g >= static_cast<uint32_t>(C::kVStages) &&
+              !(ok = warp_wait(&bars->v_empty[vs], ((g / C::kVStages) - 1) & 1)))
+            break;
+          const CUtensorMap* vmap = plane == 8 ? &maps.v8 : &maps.v4;
+          if (elect_one()) {
+            mbar_arrive_expect_tx(&bars->v_full[vs], C::kVTile);
+            if constexpr (C::kBlocksPerLoad == 1) {
+              // one block of 128 keys as two V sub-tiles of 64 keys
+              const int vrow = static_cast<int>((grp * a.nb + j0) * D);
+              tma_load_2d(sV(vs), vmap, &bars->v_full[vs], 0, vrow);
+              tma_load_2d(sV(vs) + C::kVSub, vmap, &bars->v_full[vs], 64, vrow);
+            } else {
+              const int jb[2] = {j0, j1 >= 0 ? j1 : j0};
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+                tma_load_2d(sV(vs) + h * C::kVSub, vmap, &bars->v_full[vs], 0, static_cast<int>((grp * a.nb + jb[h]) * D));
+            }
+          }
+          __syncwarp();
+          ++g;
+        }
+        if (!ok) break;
+      }
+      for (uint32_t k = (g > static_cast<uint32_t>(C::kVStages) ? g - C::kVStages : 0); k < g; ++k)
+        drain_wait(&bars->v_full[k % C::kVStages], (k / C::kVStages) & 1);
     } else if (warp == kMmaWarp) {
-      // ---------------------------------------------------------- MMA issuer
+      // ---------------------------------------------------------- QK issuer
+      // A pair's next S is computed as soon as its current S has been read out, so
+      // QK runs up to two loads ahead of P.V; the two streams are issued by two
+      // warps and meet only through the barriers.
       uint32_t g = 0, uloc = 0;
       bool ok = true;
       const uint32_t q8a = smem_u32(sQ8), q4a = smem_u32(sQ4);
-      // P.V of load gg into the O accumulator of its parity; `first` overwrites.
-      auto pv = [&](uint32_t gg, bool first) -> bool {
-        const int st = gg % C::kStages, sl = gg % C::kSlots, acc = gg % kPairs;
-        const uint32_t vbase = smem_u32(sV(st));
-        if (!warp_wait(&bars->p_full[sl], (gg / C::kSlots) & 1)) return false;
-        tc_fence_after();
-        const uint64_t vdesc = sw128_desc(vbase);
-        if (elect_one()) {
-#pragma unroll
-          for (int s = 0; s < kKeys / 16; ++s) {
-            // +((s / 4) * sub-tile + (s % 4) * 32 bytes) in the descriptor's 16-byte units
-            const uint64_t bdesc = vdesc + static_cast<uint64_t>(((s / 4) * C::kVSub + (s % 4) * 32) >> 4);
-            mma_bf16_ts(tmem + o_col(acc), tmem + sl * kKeys + s * 8, bdesc, C::kIdescPV, (first && s == 0) ? 0u : 1u);
-          }
-          mma_commit(&bars->kv_empty[st]);
-        }
-        __syncwarp();
-        return true;
-      };
       for (;; ++uloc) {
         const int r = uloc % kUnitRing;
         if (!(ok = warp_wait(&bars->unit_ready[r], (uloc / kUnitRing) & 1))) break;
         if (__shfl_sync(0xffffffffu, bars->unit_w[r], 0) < 0) break;   // no more tiles
-        const int qb = uloc & 1;
-        if (!(ok = warp_wait(&bars->q_full[qb], (uloc >> 1) & 1))) break;
-        tc_fence_after();
-        const uint32_t qoff = static_cast<uint32_t>(qb * 2 * C::kQTile);
-        int l = 0;
-        bool used[kPairs] = {false, false};   // accumulator written in this tile yet?
-        auto pv_next = [&](uint32_t gg) -> bool {
-          const bool first = !used[gg % kPairs];
-          used[gg % kPairs] = true;
-          return pv(gg, first);
-        };
-        // order: QK(g), then P.V(g - kLead): QK runs kLead loads ahead
+        if (!(ok = warp_wait(&bars->q_full, uloc & 1))) break;
         bool last = false;
         while (!last) {
-          const int st = g % C::kStages, sl = g % C::kSlots;
-          if (!(ok = warp_wait(&bars->kv_full[st], (g / C::kStages) & 1))) break;
+          const int ks = g % C::kKStages, sl = g % C::kSlots;
+          if (!(ok = warp_wait(&bars->k_full[ks], (g / C::kKStages) & 1))) break;
           // broadcast through a shuffle and a vote, so that the compiler sees the
           // loop, its counters and every operand derived from them as warp-uniform
-          const int4 inf = bars->info[st];
+          const int4 inf = bars->k_info[ks];
           const int plane = __shfl_sync(0xffffffffu, inf.z & 0xff, 0);
           last = __all_sync(0xffffffffu, (inf.z & kLastLoad) != 0);
-          // The slot's previous S and P belonged to load g - kSlots, whose P.V was
-          // issued before this QK by this thread: tcgen05.mma operations of one
-          // thread execute in issue order, so that P.V has read P before this QK
-          // writes the slot, and no wait is needed here.
+          // the slot's previous S (load g - 2) has been read out by its pair
+          if (g >= static_cast<uint32_t>(C::kSlots) &&
+              !(ok = warp_wait(&bars->s_free[sl], ((g / C::kSlots) - 1) & 1)))
+            break;
           tc_fence_after();
-          const uint32_t abase = (plane == 8 ? q8a : q4a) + qoff;
-          const uint32_t bbase = smem_u32(sK(st));
-          const uint64_t adesc = sw128_desc(abase), bdesc = sw128_desc(bbase);
+          const uint32_t abase = plane == 8 ? q8a : q4a;
+          const uint64_t adesc = sw128_desc(abase), bdesc = sw128_desc(smem_u32(sK(ks)));
           if (elect_one()) {
 #pragma unroll
             for (int k = 0; k < kQKRowBytes / 32; ++k)   // +32 bytes along K = +2 descriptor units
@@ -550,25 +591,58 @@ __global__ void __launch_bounds__(kThreads, 1)
               else
                 mma_f8_ss(tmem + sl * kKeys, adesc + 2 * k, bdesc + 2 * k, C::kIdescQK4, k > 0 ? 1u : 0u);
             mma_commit(&bars->s_full[sl]);
+            mma_commit(&bars->k_empty[ks]);
+            // the tile's last QK has read the Q buffer: the producer may refill it
+            if (last) mma_commit(&bars->q_empty);
           }
           __syncwarp();
-          // the tile's last QK has read its Q buffer: the producer may refill it
-          if (last && elect_one()) mma_commit(&bars->q_empty[qb]);
-          __syncwarp();
-          if (l >= C::kLead && !(ok = pv_next(g - C::kLead))) break;
-          ++l;
           ++g;
         }
         if (!ok) break;
-        for (int k = (l < C::kLead ? l : C::kLead); k > 0 && ok; --k) ok = pv_next(g - k);
+      }
+      // wait for every tensor-core op this warp issued before TMEM is released
+      if (elect_one()) mma_commit(&bars->fin);
+      __syncwarp();
+      drain_wait(&bars->fin, 0);
+    } else if (warp == kPvWarp) {
+      // ---------------------------------------------------------- P.V issuer
+      uint32_t g = 0, uloc = 0;
+      bool ok = true;
+      for (;; ++uloc) {
+        const int r = uloc % kUnitRing;
+        if (!(ok = warp_wait(&bars->unit_ready[r], (uloc / kUnitRing) & 1))) break;
+        if (__shfl_sync(0xffffffffu, bars->unit_w[r], 0) < 0) break;   // no more tiles
+        const int n = __shfl_sync(0xffffffffu, bars->unit_loads[r], 0);
+        for (int l = 0; l < n; ++l, ++g) {
+          const int pr = g % kPairs;   // pair = V stage = P buffer = O accumulator
+          if (!(ok = warp_wait(&bars->p_full[pr], (g / kPairs) & 1))) break;
+          if (!(ok = warp_wait(&bars->v_full[pr], (g / kPairs) & 1))) break;
+          tc_fence_after();
+          const uint64_t pdesc = sw128_desc(smem_u32(sP(pr)));
+          const uint64_t vdesc = sw128_desc(smem_u32(sV(pr)));
+          // the first P.V of a tile into an accumulator overwrites it: the tile's
+          // loads l = 0 and l = 1 are the first of their pairs
+          const bool first = l < kPairs;
+          if (elect_one()) {
+#pragma unroll
+            for (int s = 0; s < kKeys / 16; ++s) {
+              // +((s / 4) * sub-tile + (s % 4) * 32 bytes) in the descriptor's 16-byte units
+              const uint64_t adv = static_cast<uint64_t>((s % 4) * 32 >> 4);
+              const uint64_t ad = pdesc + adv + static_cast<uint64_t>(((s / 4) * C::kPSub) >> 4);
+              const uint64_t bd = vdesc + adv + static_cast<uint64_t>(((s / 4) * C::kVSub) >> 4);
+              mma_bf16_ss(tmem + o_col(pr), ad, bd, C::kIdescPV, (first && s == 0) ? 0u : 1u);
+            }
+            mma_commit(&bars->v_empty[pr]);
+          }
+          __syncwarp();
+        }
         if (!ok) break;
         if (elect_one()) mma_commit(&bars->o_fin);
         __syncwarp();
       }
-      // wait for every tensor-core op this CTA issued before TMEM is released
-      if (elect_one()) mma_commit(&bars->fin);
+      if (elect_one()) mma_commit(&bars->fin_pv);
       __syncwarp();
-      drain_wait(&bars->fin, 0);
+      drain_wait(&bars->fin_pv, 0);
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
@@ -580,19 +654,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = sub * 32 + lane;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(sub * 32) << 16);
     const uint32_t my_s = lane_addr + half * TH;                     // + slot * kKeys: S columns of my keys
-    const uint32_t my_p = lane_addr + half * (TH / 2);               // + slot * kKeys: P words of my keys
     const uint32_t my_o = lane_addr + o_col(pair) + half * (D / 2);  // O columns rescaled here
     const uint32_t pair_bar = 1 + pair * 4 + sub;                    // 64 threads: this row's pair
     const uint32_t row_bar = 9 + sub;                                // 128 threads: all four of the row
     // row maxima of loads: [pair][half][row]; epilogue (m, l): [tile parity][pair][half][2][row]
     float* xmax = reinterpret_cast<float*>(smem + C::kOffX);
     float* xepi = xmax + 2 * 2 * 128;
+    // Every wait below is shared with the warps that meet this one in a named
+    // barrier (the pair's other half per load, the row's four warps per tile): all
+    // wait on the same phases and give up only at the time limit (mbar_wait_shared),
+    // so a failure makes them leave at the same point and none is left in a barrier.
+    auto wait = [&](uint64_t* bar, uint32_t parity) { return mbar_wait_shared(bar, parity, abort, a.err); };
     uint32_t g = 0, uloc = 0;
     bool ok = true;
     for (;; ++uloc) {
       // the CTA's next tile and its load count, published by the producer
       const int r = uloc % kUnitRing;
-      if (!(ok = mbar_wait(&bars->unit_ready[r], (uloc / kUnitRing) & 1, abort, a.err))) break;
+      if (!(ok = wait(&bars->unit_ready[r], (uloc / kUnitRing) & 1))) break;
       const int w = bars->unit_w[r];
       if (w < 0) break;                                 // no more tiles
       const Unit u = unit_of(a, w, C::kQBlocks);
@@ -605,24 +683,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float a4 = valid ? a.q4s[qrow] * a.qk_log2 : 0.0f;
       const int hi = a.hi[u.hq], keep = a.keep[u.hq];
       float m_run = -INFINITY, l_run = 0.0f;     // m_run: shared by both halves of the pair
-      int64_t g_mine = -1;                        // last load of this tile handled by this pair
       // this tile's loads are g0 .. g0 + n - 1 in the CTA's order; the pair takes
       // those of its parity
       const uint32_t g0 = g, g_end = g0 + static_cast<uint32_t>(bars->unit_loads[r]);
       for (g = g0 + ((g0 % kPairs) == static_cast<uint32_t>(pair) ? 0u : 1u); g < g_end; g += kPairs) {
-        const int st = g % C::kStages, sl = g % C::kSlots;
+        const int sc = g % C::kScStages, sl = g % C::kSlots;   // sl = pair
         const uint32_t slot_col = static_cast<uint32_t>(sl * kKeys);
-        if (!(ok = mbar_wait(&bars->kv_full[st], (g / C::kStages) & 1, abort, a.err))) break;
-        if (!(ok = mbar_wait(&bars->s_full[sl], (g / C::kSlots) & 1, abort, a.err))) break;
+        if (!(ok = wait(&bars->sc_full[sc], (g / C::kScStages) & 1))) break;
+        if (!(ok = wait(&bars->s_full[sl], (g / C::kSlots) & 1))) break;
         tc_fence_after();
-        const int4 inf = bars->info[st];
+        const int4 inf = bars->sc_info[sc];
         const int plane = inf.z & 0xff;
         // my keys: a half of the load's block at T = 128; at T = 64 the block of my
         // half (j1 < 0: none, the half holds a masked copy)
         const int jh = (C::kBlocksPerLoad == 1 || half == 0) ? inf.x : inf.y;
         const int koff = C::kBlocksPerLoad == 1 ? half * TH : 0;   // my first key inside block jh
-        const bool had_prev = g_mine >= 0;        // this pair's previous load (g - 2) is in this tile
-        g_mine = g;
         // rows whose tile with block jh has another action (or none) write P = 0;
         // uniform over the warp (its 32 rows are in one query block)
         const int act = (valid && jh >= 0) ? tile_action(ir, jh, hi, keep) : ACT_NONE;
@@ -631,10 +706,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kmax = (jh == ir) ? rl - koff : TH;   // my keys [0, kmax] are visible
         float* xb = xmax + pair * 256;
         // Both halves exchange their maxima on every load (an inactive half offers
-        // -inf) and take the same decision on the running maximum. Each half has
-        // read its S (tcgen05.wait::ld) before the barrier, so no P is stored over
-        // an S that the other half has yet to read.
-        float sc = 1.0f;
+        // -inf) and take the same decision on the running maximum. Before writing
+        // its maximum a half waits for the pair's previous P.V (below), which needed
+        // the other half's previous P, written after that half read the last
+        // exchange: one buffer is enough.
+        float sc_o = 1.0f;
         bool rescale_o = false;
         auto exchange = [&](float m_half) {
           xb[half * 128 + row] = m_half;
@@ -642,74 +718,82 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float mt = fmaxf(m_half, xb[(1 - half) * 128 + row]);
           const float m_tile = mt == -INFINITY ? -INFINITY : mt * alpha;
           const bool raise = m_tile > m_run + kRescaleLog2;
-          sc = raise ? fast_exp2(m_run - m_tile) : 1.0f;
+          sc_o = raise ? fast_exp2(m_run - m_tile) : 1.0f;
           rescale_o = raise && m_run != -INFINITY;
           if (raise) {
-            l_run *= sc;
+            l_run *= sc_o;
             m_run = m_tile;
           }
         };
+        // The pair's S slot is released as soon as S is in registers, so the QK of
+        // the pair's next load runs while this one is being processed; the scales
+        // are released after the pass that reads them.
+        auto release = [&](uint64_t* bar) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar);
+        };
+        // The P.V of this pair's previous load (g - 2) reads this pair's P buffer and
+        // writes its O accumulator: it must be complete before either is touched.
+        // Its completion is phase (g / 2 - 1) of the pair's V stage barrier, which
+        // cannot have run further ahead (the next phase needs this load's P).
+        auto wait_prev_pv = [&]() -> bool {
+          return g < static_cast<uint32_t>(kPairs) || wait(&bars->v_empty[sl], ((g / kPairs) - 1) & 1);
+        };
+        // my 128-byte row of the pair's P sub-tile `half` (K-major, 128-byte swizzle)
+        uint8_t* prow = sP(pair) + half * C::kPSub + row * 128;
         if (active) {
-          uint32_t r[TH];
+          uint32_t rr[TH];
 #pragma unroll
           for (int c = 0; c < TH / 32; ++c)
-            tmem_ld32(my_s + slot_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
-          const float* sk = sScale(st) + half * TH;
+            tmem_ld32(my_s + slot_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&rr[32 * c]));
           tmem_wait_ld();
+          tc_fence_before();
+          release(&bars->s_free[sl]);
+          const float* sk = sScale(sc) + half * TH;
           uint64_t y[TH / 2];
           const bool masked = kmax < TH - 1;
           float mh;
-          if (plane == 8) mh = masked ? scores_and_max<TH, true, false>(r, y, sk, kmax) : scores_and_max<TH, false, false>(r, y, sk, kmax);
-          else mh = masked ? scores_and_max<TH, true, true>(r, y, sk, kmax) : scores_and_max<TH, false, true>(r, y, sk, kmax);
+          if (plane == 8) mh = masked ? scores_and_max<TH, true, false>(rr, y, sk, kmax) : scores_and_max<TH, false, false>(rr, y, sk, kmax);
+          else mh = masked ? scores_and_max<TH, true, true>(rr, y, sk, kmax) : scores_and_max<TH, false, true>(rr, y, sk, kmax);
+          release(&bars->sc_empty[sc]);
+          if (!(ok = wait_prev_pv())) break;
           exchange(mh);
           const uint64_t al2 = pk2(alpha, alpha), nm2 = pk2(-m_run, -m_run);
           uint64_t acc[4] = {0, 0, 0, 0};
-          {
-            uint32_t pk[TH / 2];
-            if (masked) probs<TH, true>(y, al2, nm2, kmax, pk, acc);
-            else probs<TH, false>(y, al2, nm2, kmax, pk, acc);
-            tmem_store_words<TH / 2>(my_p + slot_col, pk);
-          }
+          if (masked) probs<TH, true>(y, al2, nm2, kmax, prow, row & 7, acc);
+          else probs<TH, false>(y, al2, nm2, kmax, prow, row & 7, acc);
           float s0, s1;
           up2(add2(add2(acc[0], acc[1]), add2(acc[2], acc[3])), s0, s1);
           l_run += s0 + s1;
         } else {
-          exchange(-INFINITY);
-          uint32_t z[TH / 2];
-#pragma unroll
-          for (int k = 0; k < TH / 2; ++k) z[k] = 0u;
-          tmem_store_words<TH / 2>(my_p + slot_col, z);
-        }
-        {
-          // Rescale this half's O columns when the maximum rose (before P.V of this load
-          // may start). TMEM loads/stores are warp-collective: the whole warp takes part
-          // when any lane must, lanes that need not using the factor 1.
-          if (__any_sync(0xffffffffu, rescale_o)) {
-            // P.V of this pair's previous load (g - 2) writes this accumulator: it
-            // must be complete. With kLead = 1 the completed QK of this load implies
-            // it; with kLead = 2 it may still run. Its stage's kv_empty is then at
-            // most one phase short of it: the stage's next load is g - 2 + kStages.
-            if (C::kLead > 1 && had_prev) {
-              const uint32_t gp = g - 2;
-              if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars->kv_empty[gp % C::kStages],
-                                                           (gp / C::kStages) & 1, abort, a.err))))
-                break;
-            }
-            tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < D / 64; ++c) {
-              uint32_t o[32];
-              tmem_ld32(my_o + 32 * c, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * sc);
-              tmem_st32(my_o + 32 * c, o);
-            }
+          if (lane == 0) {
+            mbar_arrive(&bars->s_free[sl]);
+            mbar_arrive(&bars->sc_empty[sc]);
           }
+          if (!(ok = wait_prev_pv())) break;
+          exchange(-INFINITY);
+#pragma unroll
+          for (int c = 0; c < TH / 8; ++c) *reinterpret_cast<uint4*>(prow + (c << 4)) = make_uint4(0u, 0u, 0u, 0u);
         }
-        // every lane's P is in TMEM (wait::st) and ordered before the warp barrier
-        // (fence::before_thread_sync); one lane then arrives for the warp
-        tmem_wait_st();
+        // Rescale this half's O columns when the maximum rose. TMEM loads/stores are
+        // warp-collective: the whole warp takes part when any lane must, lanes that
+        // need not using the factor 1.
+        if (__any_sync(0xffffffffu, rescale_o)) {
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            uint32_t o[32];
+            tmem_ld32(my_o + 32 * c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * sc_o);
+            tmem_st32(my_o + 32 * c, o);
+          }
+          tmem_wait_st();
+        }
+        // P (generic-proxy stores) must be visible to the tensor core's reads, and a
+        // rescaled O complete (wait::st above), before the warp's one arrival
+        fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->p_full[sl]);
@@ -719,7 +803,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Epilogue: every P.V of this tile has completed (o_fin, one phase per tile; the
       // next tile's first P.V needs a P from after this epilogue, so the barrier is at
       // most one phase short).
-      if (!(ok = mbar_wait(&bars->o_fin, uloc & 1, abort, a.err))) break;
+      if (!(ok = wait(&bars->o_fin, uloc & 1))) break;
       tc_fence_after();
       float* xe = xepi + (uloc & 1) * (2 * 2 * 2 * 128);
       auto slot = [&](int p, int h, int v) { return xe + ((p * 2 + h) * 2 + v) * 128 + row; };
