@@ -13,10 +13,13 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "load_plan.cuh"
 #include "tria.h"
 
 namespace tria {
 namespace {
+
+constexpr int kRowsPerTile = 128;   // query rows of a fused-prefill tile
 
 constexpr size_t kAlign = 256;
 
@@ -266,6 +269,35 @@ int tria_count_tiles(int nb, int hi, int keep, int64_t* out) {
       const int a = tile_action(i, j, hi, keep);
       if (a == ACT_INT8) ++out[0]; else if (a == ACT_INT4) ++out[1]; else if (a == ACT_SKIP) ++out[2];
     }
+  return TRIA_OK;
+}
+
+int tria_prefill_load_plan(int nb, int T, int hi, int keep, int32_t* plan, int64_t capacity, int64_t* count) {
+  if (count == nullptr || nb < 0 || (T != 64 && T != 128) || hi < 0 || keep < hi || capacity < 0)
+    return TRIA_ERR_INVALID_ARG;
+  const int nq = kRowsPerTile / T;
+  int64_t n = 0;
+  for (int i0 = 0; i0 < nb; i0 += nq) {
+    const int q = std::min(nq, nb - i0);
+    int j0, j1, plane;
+    auto emit = [&]() {
+      if (plan != nullptr && n < capacity) {
+        int32_t* e = plan + 4 * n;
+        e[0] = i0; e[1] = j0; e[2] = j1; e[3] = plane;
+      }
+      ++n;
+    };
+    if (T == 128) {
+      LoadPairs<1> lp;
+      lp.init(i0, q, hi, keep);
+      while (lp.next(j0, j1, plane)) emit();
+    } else {
+      LoadPairs<2> lp;
+      lp.init(i0, q, hi, keep);
+      while (lp.next(j0, j1, plane)) emit();
+    }
+  }
+  *count = n;
   return TRIA_OK;
 }
 

@@ -64,6 +64,8 @@ def lib():
         L.tria_quantize_kv.restype = I
         L.tria_count_tiles.argtypes = [I, I, I, P]
         L.tria_count_tiles.restype = I
+        L.tria_prefill_load_plan.argtypes = [I, I, I, I, P, I64, P]
+        L.tria_prefill_load_plan.restype = I
         L.tria_prefill_workspace_bytes.argtypes = [ctypes.POINTER(tria_dims)]
         L.tria_prefill_workspace_bytes.restype = SZ
         L.tria_prefill.argtypes = [P, ctypes.POINTER(tria_kv_cache), ctypes.POINTER(tria_dims), P, P, P, P, P,
@@ -171,6 +173,17 @@ def tria_count_tiles(nb: int, hi: int, keep: int):
     out = np.zeros(3, np.int64)
     _check("tria_count_tiles", lib().tria_count_tiles(nb, hi, keep, out.ctypes.data_as(ctypes.c_void_p)))
     return tuple(int(v) for v in out)
+
+
+def tria_prefill_load_plan(nb: int, T: int, hi: int, keep: int) -> np.ndarray:
+    """The fused prefill's loads for one query head: int32 [n, 4] rows of
+    (first query block of the tile, j0, j1, plane), in issue order."""
+    n = ctypes.c_int64(0)
+    _check("tria_prefill_load_plan", lib().tria_prefill_load_plan(nb, T, hi, keep, None, 0, ctypes.byref(n)))
+    out = np.zeros((n.value, 4), np.int32)
+    _check("tria_prefill_load_plan", lib().tria_prefill_load_plan(nb, T, hi, keep, out.ctypes.data_as(ctypes.c_void_p),
+                                                                  n.value, ctypes.byref(n)))
+    return out
 
 
 def tria_prefill_workspace_bytes(B, Hq, Hkv, S, D, T) -> int:

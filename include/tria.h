@@ -116,6 +116,20 @@ int tria_quantize_kv(const void* K, const void* V, int S, int start,
  * out[0] = int8 tiles, out[1] = int4 tiles, out[2] = skipped causal tiles. */
 int tria_count_tiles(int nb, int hi, int keep, int64_t* out);
 
+/* The loads the fused prefill makes for one query head (host-only helper; the
+ * kernel's producers follow the same plan). The tile action is the one of the
+ * rit.work TriAttention page, section on which links may be skipped and which
+ * must be kept, as tria_count_tiles counts it. Query tiles are 128 rows: one
+ * query block at T = 128, two at T = 64; they are listed in ascending order and
+ * each tile's loads in the order the kernel issues them. A load is 128 keys:
+ * four int32 per load, (i0, j0, j1, plane): the tile's first query block, the key
+ * blocks (j1 = j0 at T = 128; at T = 64 j1 is a second block of the same plane, or
+ * -1 when j0 goes alone) and the plane, 8 or 4.
+ * nb >= 0 blocks, T in {64, 128}, 0 <= hi <= keep. `plan` (host memory, may be
+ * NULL) receives min(count, capacity) loads; *count receives the total.
+ * Returns TRIA_ERR_INVALID_ARG on a bad argument or a NULL `count`. */
+int tria_prefill_load_plan(int nb, int T, int hi, int keep, int32_t* plan, int64_t capacity, int64_t* count);
+
 /* Workspace bytes tria_prefill needs for `dims` (0 if dims are invalid). */
 size_t tria_prefill_workspace_bytes(const tria_dims* dims);
 
