@@ -131,11 +131,11 @@ struct Bars {
   uint64_t sc_full[4], sc_empty[4];     // K scales + load info: emptied by the softmax pair
   uint64_t s_full[2], s_free[2];        // S slot written by QK / read out by the pair
   uint64_t p_full[2];                   // the pair's P buffer written
-
   uint32_t tmem_base;
   int abort;
-  // Published by the producer so that the other roles need not walk the load
-  // sequence: per K stage and per scale stage the load's key blocks and plane
+  // Published by the producer so that the QK issuer, the P.V issuer and the
+  // softmax need not walk the load sequence (the V producer walks it itself, from
+  // the same tile entries): per K stage and per scale stage the load's key blocks and plane
   // (kLastLoad marks a tile's last load), visible after the stage's full barrier;
   // per tile u of this CTA, the tile's index and load count in ring entry
   // u % kUnitRing (index -1: no more tiles), visible after phase u / kUnitRing of
