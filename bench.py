@@ -462,15 +462,19 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        vals = []
+        vals, secs = [], []
         for _ in range(args.warmup):
             oracle_sample(w, budget_s=2.0)
         for k in range(args.steps):
+            t0 = time.perf_counter()
             v, unit, note, cores = oracle_sample(w, budget_s=args.cpu_budget / max(1, args.steps), seed=k + 1)
+            secs.append(time.perf_counter() - t0)
             vals.append(v)
         v = float(np.mean(vals))
+        # n_gpus 0: this arm is the CPU oracle; a step is one bounded sample of the workload
         print(json.dumps({"impl": "reference", "metric": metric_name(w), "value": v, "unit": unit, "n_gpus": 0,
-                          "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+                          "steps": args.steps, "warmup": args.warmup,
+                          "ms_per_step": 1e3 * float(np.mean(secs)), "higher_is_better": True,
                           "scaling": "weak", "vs_baseline": None, "dtype": "f64 softmax / int codes",
                           "data": "synthetic", "config": config_of(w, args, 1),
                           "cpu_baseline": {"value": v, "unit": unit, "cores": cores, "kind": "oracle",
