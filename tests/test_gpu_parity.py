@@ -164,6 +164,27 @@ def test_prefill_llama_workload_sampled_rows(T, oracle_mod):
     compare_lse(L.reshape(-1).cpu()[idx], L_ref, "llama sampled")
 
 
+@pytest.mark.parametrize("Tb", [64, 128])
+def test_prefill_many_short_tiles_sampled_rows(T, oracle_mod, Tb):
+    """Tiles of one to three loads each, about 17 per CTA: each CTA runs through
+    its 16-entry tile ring more than once and meets every tile boundary case
+    (a tile whose only load belongs to one pair, lone blocks of either plane)."""
+    B, Hq, Hkv, S, D = 1, 16, 4, 20480, 128
+    pol = [(0, 0), (0, 1), (1, 2), (0, 2)] * 4
+    hi = np.array([p[0] for p in pol], np.int32)
+    keep = np.array([p[1] for p in pol], np.int32)
+    Q, K, V = seeded((B, Hq, S, D), 71), seeded((B, Hkv, S, D), 72), seeded((B, Hkv, S, D), 73)
+    O, L, _ = run_prefill(T, Q, K, V, Tb, hi, keep)
+    rng = np.random.RandomState(Tb)
+    picks = [(0, h, t) for h in range(Hq) for t in (0, Tb - 1, Tb, 2 * Tb + 5, S - 1)]
+    picks += [(0, int(rng.randint(Hq)), int(rng.randint(S))) for _ in range(384)]
+    rows = rows_of(B, Hq, S, picks)
+    O_ref, L_ref = oracle_mod.prefill_rows(Q, K, V, Tb, hi, keep, rows=rows)
+    idx = torch.from_numpy(rows)
+    compare_o(O.reshape(-1, D).cpu()[idx], O_ref, f"short tiles T{Tb}")
+    compare_lse(L.reshape(-1).cpu()[idx], L_ref, f"short tiles T{Tb}")
+
+
 def test_prefill_skipped_blocks_are_never_read(T, oracle_mod):
     """Overwrite the cache codes of one key block: rows whose tile with it is
     skipped must come out bit-identical; rows that keep it must change."""
