@@ -201,6 +201,20 @@ def decode_bytes(B, Hq, Hkv, D, T, kv_len, hi, keep):
 
 # ---------------------------------------------------------------- GPU arm
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest x over all ranks: a job's step takes as long as its slowest rank."""
+    if world <= 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms: float) -> float:
+    """Units that all ranks processed, per second of the slowest rank's time."""
+    return units_per_rank * world / (ms / 1e3)
+
+
 def run_gpu(args, rank, world, device):
     from block_sparse_mixed_b200 import tria
     from block_sparse_mixed_b200.build import build
@@ -287,16 +301,12 @@ def run_gpu(args, rank, world, device):
     seg = np.array([[times[k][i].elapsed_time(times[k][i + 1]) for i in range(len(times[k]) - 1)]
                     for k in range(len(times))])          # ms per segment per step
     step_ms = float(seg.sum(axis=1).mean())
-    step_ms_max = step_ms
-    if world > 1:
-        t = torch.tensor([step_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        step_ms_max = float(t.item())
+    step_ms_max = max_over_ranks(step_ms, world, device)
 
     res = {"clocks": clk.summary(), "ms_per_step": step_ms_max}
     if w.kind == "prefill":
         tokens = w.B * w.S
-        res["value"] = tokens * world / (step_ms_max / 1e3)
+        res["value"] = whole_job_rate(tokens, world, step_ms_max)
         q_ms, prep_ms, att_ms, d_ms = (float(seg[:, i].mean()) for i in range(4))
         p_ms = prep_ms + att_ms
         p_i8 = peaks["bf16_tflops"] * INT8_OVER_BF16
@@ -322,7 +332,7 @@ def run_gpu(args, rank, world, device):
     else:
         d_ms = float(seg[:, 0].mean())
         gbs = dbytes / (d_ms / 1e3) / 1e9
-        res["value"] = gbs * world
+        res["value"] = whole_job_rate(dbytes, world, step_ms_max) / 1e9
         res["roofline"] = {"bound": "hbm", "kernel": "tria_decode (decode_kernel + decode_merge_kernel)",
                            "achieved": gbs, "peak": peaks["hbm_gbs"],
                            "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
@@ -372,15 +382,11 @@ def run_gpu(args, rank, world, device):
         b.record(stream)
         b.synchronize()
         e_ms.append(a.elapsed_time(b))
-    e2e_ms = float(np.mean(e_ms))
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(float(np.mean(e_ms)), world, device)
     if units is not None:
-        e2e_val, e2e_unit = units * world / (e2e_ms / 1e3), "tokens/s"
+        e2e_val, e2e_unit = whole_job_rate(units, world, e2e_ms), "tokens/s"
     else:
-        e2e_val, e2e_unit = dbytes * world / (e2e_ms / 1e3) / 1e9, "GB/s"
+        e2e_val, e2e_unit = whole_job_rate(dbytes, world, e2e_ms) / 1e9, "GB/s"
     res["e2e"] = {"value": e2e_val, "unit": e2e_unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                   "ms_per_step": e2e_ms}
     return res
