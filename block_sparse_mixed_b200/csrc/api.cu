@@ -105,7 +105,28 @@ int check_cache(const tria_kv_cache* c) {
   const void* ptrs[8] = {c->k8, c->k4, c->k8_scale, c->k4_scale, c->v8, c->v4, c->v8_scale, c->v4_scale};
   for (const void* p : ptrs)
     if (p == nullptr || !aligned16(p)) return TRIA_ERR_INVALID_ARG;
+  if (c->status == nullptr) return TRIA_ERR_INVALID_ARG;
+  if (c->block_table != nullptr) {
+    if (c->max_blocks < 1 || c->num_pages < 1 || c->capacity != c->max_blocks * c->T) return TRIA_ERR_INVALID_ARG;
+    // TMA row coordinates and the page arithmetic are 32-bit
+    if (static_cast<int64_t>(c->num_pages) * c->Hkv * c->T >= (int64_t(1) << 31)) return TRIA_ERR_UNSUPPORTED;
+  } else if (static_cast<int64_t>(c->B) * c->Hkv * c->capacity >= (int64_t(1) << 31)) {
+    return TRIA_ERR_UNSUPPORTED;
+  }
   return TRIA_OK;
+}
+
+// Where the kernels find the cache's tokens.
+CacheIndex cache_index(const tria_kv_cache& c) {
+  CacheIndex ci{};
+  ci.bt = c.block_table;
+  ci.status = c.status;
+  ci.cap = c.capacity;
+  ci.Hkv = c.Hkv;
+  ci.T = c.T;
+  ci.max_blocks = c.max_blocks;
+  ci.num_pages = c.num_pages;
+  return ci;
 }
 
 int check_policy(const int32_t* hi, const int32_t* keep, int Hq) {
@@ -120,7 +141,7 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? TRIA_OK : TRIA_ERR_CU
 // ---------------------------------------------------------------- workspace layouts
 
 struct PrefillLayout {
-  size_t ctrl, q8, q4, q8s, q4s, k4x, k8x, vt8, vt4, total;
+  size_t ctrl, q8, q4, q8s, q4s, k4x, k8x, vd8, vd4, total;
 };
 
 PrefillLayout prefill_layout(const tria_dims& d) {
@@ -135,8 +156,8 @@ PrefillLayout prefill_layout(const tria_dims& d) {
   L.q4s = off; off += align_up(qrows * 4);
   L.k4x = off; off += align_up(krows * kQKRowBytes);
   L.k8x = off; if (d.D < 128) off += align_up(krows * kQKRowBytes);
-  L.vt8 = off; off += align_up(krows * d.D * 2);
-  L.vt4 = off; off += align_up(krows * d.D * 2);
+  L.vd8 = off; off += align_up(krows * d.D * 2);
+  L.vd4 = off; off += align_up(krows * d.D * 2);
   L.total = off;
   return L;
 }
@@ -196,19 +217,16 @@ const char* tria_status_string(int status) {
   }
 }
 
-size_t tria_cache_bytes(int B, int Hkv, int D, int T, int capacity) {
-  if (B < 1 || Hkv < 1 || !shape_ok(D, T) || capacity < 1 || capacity % T != 0) return 0;
-  const size_t rows = static_cast<size_t>(B) * Hkv * capacity;
-  return 2 * (align_up(rows * D) + align_up(rows * D / 2) + 2 * align_up(rows * 4));
+namespace {
+
+// Planes of `rows` token rows after a 256-byte status block, in the order of the struct.
+size_t planes_bytes(size_t rows, int D) {
+  return align_up(64) + 2 * (align_up(rows * D) + align_up(rows * D / 2) + 2 * align_up(rows * 4));
 }
 
-int tria_cache_init(tria_kv_cache* c, void* base, size_t bytes, int B, int Hkv, int D, int T, int capacity) {
-  if (c == nullptr || base == nullptr || !aligned256(base)) return TRIA_ERR_INVALID_ARG;
-  const size_t need = tria_cache_bytes(B, Hkv, D, T, capacity);
-  if (need == 0) return shape_ok(D, T) ? TRIA_ERR_INVALID_ARG : TRIA_ERR_UNSUPPORTED;
-  if (bytes < need) return TRIA_ERR_INVALID_ARG;
-  const size_t rows = static_cast<size_t>(B) * Hkv * capacity;
+void carve(tria_kv_cache* c, void* base, size_t rows, int D) {
   uint8_t* p = static_cast<uint8_t*>(base);
+  c->status = reinterpret_cast<int*>(p); p += align_up(64);
   c->k8 = reinterpret_cast<int8_t*>(p); p += align_up(rows * D);
   c->k4 = p; p += align_up(rows * D / 2);
   c->k8_scale = reinterpret_cast<float*>(p); p += align_up(rows * 4);
@@ -217,8 +235,55 @@ int tria_cache_init(tria_kv_cache* c, void* base, size_t bytes, int B, int Hkv, 
   c->v4 = p; p += align_up(rows * D / 2);
   c->v8_scale = reinterpret_cast<float*>(p); p += align_up(rows * 4);
   c->v4_scale = reinterpret_cast<float*>(p);
+}
+
+}  // namespace
+
+size_t tria_cache_bytes(int B, int Hkv, int D, int T, int capacity) {
+  if (B < 1 || Hkv < 1 || !shape_ok(D, T) || capacity < 1 || capacity % T != 0) return 0;
+  return planes_bytes(static_cast<size_t>(B) * Hkv * capacity, D);
+}
+
+int tria_cache_init(tria_kv_cache* c, void* base, size_t bytes, int B, int Hkv, int D, int T, int capacity) {
+  if (c == nullptr || base == nullptr || !aligned256(base)) return TRIA_ERR_INVALID_ARG;
+  const size_t need = tria_cache_bytes(B, Hkv, D, T, capacity);
+  if (need == 0) return shape_ok(D, T) ? TRIA_ERR_INVALID_ARG : TRIA_ERR_UNSUPPORTED;
+  if (bytes < need) return TRIA_ERR_INVALID_ARG;
+  std::memset(c, 0, sizeof *c);
+  carve(c, base, static_cast<size_t>(B) * Hkv * capacity, D);
   c->B = B; c->Hkv = Hkv; c->D = D; c->T = T; c->capacity = capacity;
   return TRIA_OK;
+}
+
+size_t tria_paged_cache_bytes(int num_pages, int Hkv, int D, int T) {
+  if (num_pages < 1 || Hkv < 1 || !shape_ok(D, T)) return 0;
+  return planes_bytes(static_cast<size_t>(num_pages) * Hkv * T, D);
+}
+
+int tria_paged_cache_init(tria_kv_cache* c, void* base, size_t bytes, int B, int Hkv, int D, int T, int num_pages,
+                          const int32_t* block_table, int max_blocks) {
+  if (c == nullptr || base == nullptr || !aligned256(base) || block_table == nullptr) return TRIA_ERR_INVALID_ARG;
+  if (!shape_ok(D, T)) return TRIA_ERR_UNSUPPORTED;
+  if (B < 1 || max_blocks < 1 || static_cast<int64_t>(max_blocks) * T >= (int64_t(1) << 31))
+    return TRIA_ERR_INVALID_ARG;
+  const size_t need = tria_paged_cache_bytes(num_pages, Hkv, D, T);
+  if (need == 0 || bytes < need) return TRIA_ERR_INVALID_ARG;
+  std::memset(c, 0, sizeof *c);
+  carve(c, base, static_cast<size_t>(num_pages) * Hkv * T, D);
+  c->B = B; c->Hkv = Hkv; c->D = D; c->T = T; c->capacity = max_blocks * T;
+  c->block_table = block_table; c->max_blocks = max_blocks; c->num_pages = num_pages;
+  return TRIA_OK;
+}
+
+int tria_cache_status(const tria_kv_cache* c, void* stream) {
+  if (c == nullptr || c->status == nullptr) return TRIA_ERR_INVALID_ARG;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return TRIA_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpy(&word, c->status, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess) return TRIA_ERR_CUDA;
+  if (cudaMemsetAsync(c->status, 0, sizeof word, st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess)
+    return TRIA_ERR_CUDA;
+  return word;
 }
 
 int tria_quantize_rows(const void* X, int64_t rows, int D, int8_t* c8, float* s8, uint8_t* c4, float* s4,
@@ -231,7 +296,7 @@ int tria_quantize_rows(const void* X, int64_t rows, int D, int8_t* c8, float* s8
   if (!device_info().ok) return TRIA_ERR_UNSUPPORTED;
   QuantArgs a{};
   a.X = static_cast<const __nv_bfloat16*>(X);
-  a.rows = rows; a.rows_per_group = rows > 0 ? rows : 1; a.group_stride = 0; a.start = 0;
+  a.rows = rows; a.cache = false;
   a.c8 = c8; a.ld8 = D; a.c4p = c4; a.c4u = nullptr; a.ld4u = 0; a.s8 = s8; a.s4 = s4;
   return cuda_status(launch_quant_rows(a, D, static_cast<cudaStream_t>(stream)));
 }
@@ -247,8 +312,9 @@ int tria_quantize_kv(const void* K, const void* V, int S, int start, const tria_
     QuantArgs a{};
     a.X = static_cast<const __nv_bfloat16*>(which == 0 ? K : V);
     a.rows = static_cast<int64_t>(cache->B) * cache->Hkv * S;
-    a.rows_per_group = S;
-    a.group_stride = cache->capacity;
+    a.cache = true;
+    a.ci = cache_index(*cache);
+    a.S = S;
     a.start = start;
     a.c8 = which == 0 ? cache->k8 : cache->v8;
     a.ld8 = cache->D;
@@ -345,7 +411,7 @@ int tria_prefill_prepare(const void* Q, const tria_kv_cache* cache, const tria_d
   // 1. Q codes, both planes, one int8 per value in 128-byte rows
   QuantArgs qa{};
   qa.X = static_cast<const __nv_bfloat16*>(Q);
-  qa.rows = qrows; qa.rows_per_group = qrows; qa.group_stride = 0; qa.start = 0;
+  qa.rows = qrows; qa.cache = false;
   qa.c8 = reinterpret_cast<int8_t*>(ws + L.q8); qa.ld8 = kQKRowBytes;
   qa.c4p = nullptr; qa.c4u = reinterpret_cast<int8_t*>(ws + L.q4); qa.ld4u = kQKRowBytes;
   qa.s8 = reinterpret_cast<float*>(ws + L.q8s); qa.s4 = reinterpret_cast<float*>(ws + L.q4s);
@@ -357,10 +423,10 @@ int tria_prefill_prepare(const void* Q, const tria_kv_cache* cache, const tria_d
   pa.v8s = cache->v8_scale; pa.v4s = cache->v4_scale;
   pa.k8x = d.D < 128 ? reinterpret_cast<int8_t*>(ws + L.k8x) : nullptr;
   pa.k4x = reinterpret_cast<int8_t*>(ws + L.k4x);
-  pa.vt8 = reinterpret_cast<__nv_bfloat16*>(ws + L.vt8);
-  pa.vt4 = reinterpret_cast<__nv_bfloat16*>(ws + L.vt4);
-  pa.cap = cache->capacity; pa.S = d.S; pa.nb = nb;
-  if (launch_prepare(pa, d.D, d.T, groups, nb, st) != cudaSuccess) return TRIA_ERR_CUDA;
+  pa.vd8 = reinterpret_cast<__nv_bfloat16*>(ws + L.vd8);
+  pa.vd4 = reinterpret_cast<__nv_bfloat16*>(ws + L.vd4);
+  pa.ci = cache_index(*cache); pa.S = d.S; pa.groups = groups;
+  if (launch_prepare(pa, d.D, st) != cudaSuccess) return TRIA_ERR_CUDA;
   return TRIA_OK;
 }
 
@@ -384,24 +450,19 @@ int tria_prefill_attend(const tria_kv_cache* cache, const tria_dims* dims, const
   bool ok = make_map(&maps.q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + L.q8, kQKRowBytes, qrows, 128, 128) &&
             make_map(&maps.q4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + L.q4, kQKRowBytes, qrows, 128, 128) &&
             make_map(&maps.k4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + L.k4x, kQKRowBytes, krows, 128, d.T) &&
-            make_map(&maps.v8, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + L.vt8, d.T,
-                     static_cast<uint64_t>(groups) * nb * d.D, 64, d.D) &&
-            make_map(&maps.v4, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + L.vt4, d.T,
-                     static_cast<uint64_t>(groups) * nb * d.D, 64, d.D);
-  int64_t cap8;
-  if (d.D == 128) {
+            make_map(&maps.v8, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + L.vd8, d.D, krows, 64, d.T) &&
+            make_map(&maps.v4, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + L.vd4, d.D, krows, 64, d.T);
+  const CacheIndex ci = cache_index(*cache);
+  if (d.D == 128)
     ok = ok && make_map(&maps.k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, cache->k8, 128,
-                        static_cast<uint64_t>(groups) * cache->capacity, 128, d.T);
-    cap8 = cache->capacity;
-  } else {
+                        static_cast<uint64_t>(ci.rows(cache->B)), 128, d.T);
+  else
     ok = ok && make_map(&maps.k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + L.k8x, kQKRowBytes, krows, 128, d.T);
-    cap8 = d.S;
-  }
   if (!ok) return TRIA_ERR_CUDA;
 
   PrefillArgs a{};
   a.B = d.B; a.Hq = d.Hq; a.Hkv = d.Hkv; a.S = d.S; a.G = d.Hq / d.Hkv; a.nb = nb;
-  a.cap = cache->capacity; a.cap8 = cap8;
+  a.ci = ci; a.k8_in_cache = d.D == 128;
   a.n_qtiles = (d.S + 127) / 128;
   a.n_units = d.B * d.Hq * a.n_qtiles;
   a.qk_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d.D)));
@@ -483,7 +544,7 @@ int tria_decode(const void* q, const tria_kv_cache* cache, const int32_t* kv_len
 
   DecodeArgs a{};
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.G = G; a.D = D; a.T = T;
-  a.cap = cache->capacity;
+  a.ci = cache_index(*cache);
   a.blocks_per_split = bps;
   a.qk_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
   a.q = static_cast<const __nv_bfloat16*>(q);
@@ -506,8 +567,7 @@ int tria_decode(const void* q, const tria_kv_cache* cache, const int32_t* kv_len
   a.n_items = items;
 
   DecodeMaps maps;
-  const uint64_t rows = static_cast<uint64_t>(groups) * cache->capacity;
-  if (rows > static_cast<uint64_t>(INT32_MAX)) return TRIA_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
+  const uint64_t rows = static_cast<uint64_t>(a.ci.rows(B));   // below 2^31 (check_cache)
   const bool ok = make_map(&maps.k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, cache->k8, D, rows, D, T) &&
                   make_map(&maps.k4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, cache->k4, D / 2, rows, D / 2, T) &&
                   make_map(&maps.v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, cache->v8, D, rows, D, T) &&

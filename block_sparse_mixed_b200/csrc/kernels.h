@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "tria.h"
+
 namespace tria {
 
 constexpr int kMaxHeads = 256;     // Hq limit (policy arrays travel in kernel parameters)
@@ -14,13 +16,41 @@ constexpr int kMaxGroups = 2048;   // decode: B * Hkv
 constexpr int kQKRowBytes = 128;   // Q/K code rows as the tensor cores read them (D padded to 128)
 constexpr int kDecodeSlices = 8;   // decode: most compute warps per CTA (each writes its own partial)
 
-// Codec over rows. Output row of input row r:
-//   (r / rows_per_group) * group_stride + start + r % rows_per_group.
+// Where the cache keeps the tokens of one (sequence b, KV head): the contiguous
+// layout [B, Hkv, cap] rows, or pages of T tokens x Hkv heads named by a block
+// table. A page id outside [0, num_pages) sets TRIA_ERR_BOUNDS in the cache's
+// status word and gives -1; callers then skip or redirect the access.
+struct CacheIndex {
+  const int32_t* bt;      // device [B, max_blocks] page of each logical block, or null (contiguous)
+  int* status;            // the cache's device error word
+  int64_t cap;            // contiguous: tokens per (b, kv head)
+  int Hkv, T, max_blocks, num_pages;
+
+  // Cache row of the first token of logical block j of (b, kvh).
+  __device__ __forceinline__ int64_t block_row(int b, int kvh, int j) const {
+    if (bt == nullptr) return (static_cast<int64_t>(b) * Hkv + kvh) * cap + static_cast<int64_t>(j) * T;
+    const int p = (j >= 0 && j < max_blocks) ? bt[static_cast<int64_t>(b) * max_blocks + j] : -1;
+    if (p < 0 || p >= num_pages) {
+      atomicExch(status, TRIA_ERR_BOUNDS);
+      return -1;
+    }
+    return (static_cast<int64_t>(p) * Hkv + kvh) * T;
+  }
+  // Rows of one plane of the cache.
+  __host__ __device__ int64_t rows(int B) const {
+    return bt == nullptr ? static_cast<int64_t>(B) * Hkv * cap : static_cast<int64_t>(num_pages) * Hkv * T;
+  }
+};
+
+// Codec over rows. Output row of input row r: r itself (tokens of Q, or any rows),
+// or, when `cache` is set, the cache row of token start + r % S of (b, kvh) =
+// (r / S) / Hkv, (r / S) % Hkv.
 struct QuantArgs {
   const __nv_bfloat16* X;
   int64_t rows;
-  int64_t rows_per_group;
-  int64_t group_stride;
+  bool cache;
+  CacheIndex ci;
+  int64_t S;
   int64_t start;
   int8_t* c8;
   int ld8;            // bytes per c8 row (D or 128; bytes past D are zeroed)
@@ -40,17 +70,17 @@ struct PrepareArgs {
   const float* v4s;
   int8_t* k8x;        // null when D == 128 (the cache plane is read directly)
   int8_t* k4x;        // [groups * S, 128]
-  __nv_bfloat16* vt8; // [groups * nb, D, T]
-  __nv_bfloat16* vt4;
-  int64_t cap;        // cache tokens per (b, kv head)
+  __nv_bfloat16* vd8; // [groups * S, D] V of the 8-bit plane, dequantised
+  __nv_bfloat16* vd4; // [groups * S, D] V of the 4-bit plane, dequantised
+  CacheIndex ci;
   int64_t S;          // prefill tokens per (b, kv head) (= nb * T)
-  int64_t nb;
+  int64_t groups;     // B * Hkv
 };
 
 struct PrefillArgs {
   int B, Hq, Hkv, S, G, nb;
-  int64_t cap;            // cache rows per (b, kv head): scale arrays
-  int64_t cap8;           // rows per (b, kv head) behind the 8-bit K map (cap, or S when padded)
+  CacheIndex ci;          // cache rows of the 8-bit K plane (D = 128) and of the K scales
+  bool k8_in_cache;       // the 8-bit K map covers the cache plane (D = 128) or the padded copy (D = 64)
   int n_qtiles, n_units;
   float qk_log2;          // log2(e) / sqrt(D)
   const float* q8s;       // [B*Hq*S]
@@ -75,7 +105,7 @@ struct DecodeMaps {
 
 struct DecodeArgs {
   int B, Hq, Hkv, G, D, T;
-  int64_t cap;
+  CacheIndex ci;
   int n_items;            // (group, split) work items
   int blocks_per_split;
   float qk_log2;
@@ -100,7 +130,7 @@ struct DecodeArgs {
 };
 
 cudaError_t launch_quant_rows(const QuantArgs& a, int D, cudaStream_t stream);
-cudaError_t launch_prepare(const PrepareArgs& a, int D, int T, int groups, int nblocks, cudaStream_t stream);
+cudaError_t launch_prepare(const PrepareArgs& a, int D, cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillArgs& a, const PrefillMaps& maps, int D, int T, int num_sms,
                            cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, const DecodeMaps& maps, int num_sms, cudaStream_t stream);

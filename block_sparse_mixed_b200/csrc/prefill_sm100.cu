@@ -30,9 +30,10 @@
 //               as the pair has read S into registers, so the next S of a pair is
 //               computed while the pair still works on the current one.
 //   warp 18     producer of the V tiles (a ring of 2 stages, one per pair).
-//   warp 19     P.V issuer: O += P.V on kind::f16, bf16 P and V from shared memory,
-//               fp32 O in TMEM; each P.V frees its V stage, P buffer and the
-//               accumulator for the pair's next load.
+//   warp 19     P.V issuer: O += P.V on kind::f16, bf16 P (K-major) and V (N-major,
+//               the dequantised rows as they lie in memory) from shared memory, fp32 O
+//               in TMEM; each P.V frees its V stage, P buffer and the accumulator for
+//               the pair's next load.
 // Each ring is released as soon as its contents are used (K by the QK's
 // completion, the scales after the softmax's first pass, V and P by the P.V's
 // completion), so no stage is held across another role's round trip.
@@ -86,8 +87,8 @@ struct Cfg {
   static constexpr int kBlocksPerLoad = kKeys / T;           // key blocks per load
   static constexpr int kQTile = kRows * kQKRowBytes;         // Q codes of one plane
   static constexpr int kKTile = kKeys * kQKRowBytes;         // K codes of one load
-  static constexpr int kVSub = D * 128;                      // one V sub-tile: D rows x 64 keys
-  static constexpr int kVTile = D * kKeys * 2;               // both V sub-tiles of a load
+  static constexpr int kVChunk = kKeys * 128;                // V of one load, 64 values of d: 128 key rows x 128 B
+  static constexpr int kVTile = D * kKeys * 2;               // V of one load: D / 64 chunks
   static constexpr int kPSub = kRows * 128;                  // one P sub-tile: 128 rows x 64 keys
   static constexpr int kPTile = kRows * kKeys * 2;           // P of one load (bf16)
   static constexpr int kScTile = kKeys * 4;                  // K scales of one load
@@ -113,11 +114,11 @@ struct Cfg {
   static constexpr int kSmem = kSmemNeed > 120 * 1024 ? kSmemNeed : 120 * 1024;
   static_assert(kSmemNeed <= 227 * 1024, "shared memory");
   static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0 && kKTile % 1024 == 0 &&
-                    kVSub % 1024 == 0 && kPSub % 1024 == 0,
+                    kVChunk % 1024 == 0 && kPSub % 1024 == 0,
                 "swizzled operand tiles start on 1024-byte boundaries");
   static constexpr uint32_t kIdescQK = idesc_i8(kRows, kKeys);       // 8-bit plane: int8, int32 S
   static constexpr uint32_t kIdescQK4 = idesc_e4m3(kRows, kKeys);    // 4-bit plane: e4m3, fp32 S (exact)
-  static constexpr uint32_t kIdescPV = idesc_bf16(kRows, D);
+  static constexpr uint32_t kIdescPV = idesc_bf16_bn(kRows, D);     // P K-major, V N-major
 };
 
 constexpr int kUnitRing = 16;           // tiles published ahead of the consumers
@@ -405,8 +406,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           ++k_load;
           const CUtensorMap* kmap = plane == 8 ? &maps.k8 : &maps.k4;
-          const int64_t krow_base = grp * (plane == 8 ? a.cap8 : static_cast<int64_t>(a.S));
-          const float* ks_base = (plane == 8 ? a.k8s : a.k4s) + grp * a.cap;
+          const bool k_in_cache = plane == 8 && a.k8_in_cache;    // else a workspace copy, [group][S] rows
+          const float* ks_plane = plane == 8 ? a.k8s : a.k4s;
           if (elect_one()) {
             const int4 inf = make_int4(j0, j1, plane | (k_load == n_loads ? kLastLoad : 0), 0);
             bars->k_info[ks] = inf;    // released by the arrives below
@@ -418,9 +419,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int jb[2] = {j0, (C::kBlocksPerLoad == 1 || j1 < 0) ? j0 : j1};
 #pragma unroll
             for (int h = 0; h < C::kBlocksPerLoad; ++h) {
-              tma_load_2d(sK(ks) + h * T * kQKRowBytes, kmap, &bars->k_full[ks], 0,
-                          static_cast<int>(krow_base + static_cast<int64_t>(jb[h]) * T));
-              bulk_load(sScale(ss) + h * T, ks_base + static_cast<int64_t>(jb[h]) * T, T * 4, &bars->sc_full[ss]);
+              // the block's cache row (contiguous or paged; a bad page id reads page 0, reported)
+              int64_t crow = a.ci.block_row(u.b, u.kvh, jb[h]);
+              crow = crow < 0 ? 0 : crow;
+              const int64_t krow = k_in_cache ? crow : grp * a.S + static_cast<int64_t>(jb[h]) * T;
+              tma_load_2d(sK(ks) + h * T * kQKRowBytes, kmap, &bars->k_full[ks], 0, static_cast<int>(krow));
+              bulk_load(sScale(ss) + h * T, ks_plane + crow, T * 4, &bars->sc_full[ss]);
             }
           }
           __syncwarp();
@@ -458,17 +462,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const CUtensorMap* vmap = plane == 8 ? &maps.v8 : &maps.v4;
           if (elect_one()) {
             mbar_arrive_expect_tx(&bars->v_full[vs], C::kVTile);
-            if constexpr (C::kBlocksPerLoad == 1) {
-              // one block of 128 keys as two V sub-tiles of 64 keys
-              const int vrow = static_cast<int>((grp * a.nb + j0) * D);
-              tma_load_2d(sV(vs), vmap, &bars->v_full[vs], 0, vrow);
-              tma_load_2d(sV(vs) + C::kVSub, vmap, &bars->v_full[vs], 64, vrow);
-            } else {
-              const int jb[2] = {j0, j1 >= 0 ? j1 : j0};
+            // V rows [token][d] as chunks of 64 values of d, each chunk 128 key rows (the
+            // load's block, or its two blocks at T = 64, a lone block copied twice)
+            const int jb[2] = {j0, (C::kBlocksPerLoad == 1 || j1 < 0) ? j0 : j1};
 #pragma unroll
-              for (int h = 0; h < 2; ++h)
-                tma_load_2d(sV(vs) + h * C::kVSub, vmap, &bars->v_full[vs], 0, static_cast<int>((grp * a.nb + jb[h]) * D));
-            }
+            for (int c = 0; c < D / 64; ++c)
+#pragma unroll
+              for (int h = 0; h < C::kBlocksPerLoad; ++h)
+                tma_load_2d(sV(vs) + c * C::kVChunk + h * T * 128, vmap, &bars->v_full[vs], 64 * c,
+                            static_cast<int>(grp * a.S + static_cast<int64_t>(jb[h]) * T));
           }
           __syncwarp();
           ++g;
@@ -542,17 +544,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = warp_wait(&bars->v_full[pr], (g / kPairs) & 1))) break;
           tc_fence_after();
           const uint64_t pdesc = sw128_desc(smem_u32(sP(pr)));
-          const uint64_t vdesc = sw128_desc(smem_u32(sV(pr)));
+          const uint64_t vdesc = sw128_mn_desc(smem_u32(sV(pr)), C::kVChunk);
           // the first P.V of a tile into an accumulator overwrites it: the tile's
           // loads l = 0 and l = 1 are the first of their pairs
           const bool first = l < kPairs;
           if (elect_one()) {
 #pragma unroll
             for (int s = 0; s < kKeys / 16; ++s) {
-              // +((s / 4) * sub-tile + (s % 4) * 32 bytes) in the descriptor's 16-byte units
-              const uint64_t adv = static_cast<uint64_t>((s % 4) * 32 >> 4);
-              const uint64_t ad = pdesc + adv + static_cast<uint64_t>(((s / 4) * C::kPSub) >> 4);
-              const uint64_t bd = vdesc + adv + static_cast<uint64_t>(((s / 4) * C::kVSub) >> 4);
+              // P (K-major): +((s / 4) * sub-tile + (s % 4) * 32 bytes); V (N-major): + 16 key
+              // rows of 128 bytes; in the descriptors' 16-byte units
+              const uint64_t ad = pdesc + static_cast<uint64_t>((s % 4) * 32 >> 4) +
+                                  static_cast<uint64_t>(((s / 4) * C::kPSub) >> 4);
+              const uint64_t bd = vdesc + static_cast<uint64_t>((s * 16 * 128) >> 4);
               mma_bf16_ss(tmem + o_col(pr), ad, bd, C::kIdescPV, (first && s == 0) ? 0u : 1u);
             }
             mma_commit(&bars->v_empty[pr]);

@@ -33,7 +33,8 @@ class tria_kv_cache(ctypes.Structure):
                 ("k4_scale", ctypes.c_void_p), ("v8", ctypes.c_void_p), ("v4", ctypes.c_void_p),
                 ("v8_scale", ctypes.c_void_p), ("v4_scale", ctypes.c_void_p),
                 ("B", ctypes.c_int), ("Hkv", ctypes.c_int), ("D", ctypes.c_int), ("T", ctypes.c_int),
-                ("capacity", ctypes.c_int)]
+                ("capacity", ctypes.c_int), ("block_table", ctypes.c_void_p), ("max_blocks", ctypes.c_int),
+                ("num_pages", ctypes.c_int), ("status", ctypes.c_void_p)]
 
 
 class tria_dims(ctypes.Structure):
@@ -58,6 +59,12 @@ def lib():
         L.tria_cache_bytes.restype = SZ
         L.tria_cache_init.argtypes = [ctypes.POINTER(tria_kv_cache), P, SZ, I, I, I, I, I]
         L.tria_cache_init.restype = I
+        L.tria_paged_cache_bytes.argtypes = [I, I, I, I]
+        L.tria_paged_cache_bytes.restype = SZ
+        L.tria_paged_cache_init.argtypes = [ctypes.POINTER(tria_kv_cache), P, SZ, I, I, I, I, I, P, I]
+        L.tria_paged_cache_init.restype = I
+        L.tria_cache_status.argtypes = [ctypes.POINTER(tria_kv_cache), P]
+        L.tria_cache_status.restype = I
         L.tria_quantize_rows.argtypes = [P, I64, I, P, P, P, P, P]
         L.tria_quantize_rows.restype = I
         L.tria_quantize_kv.argtypes = [P, P, I, I, ctypes.POINTER(tria_kv_cache), P]
@@ -124,28 +131,60 @@ def _aligned_empty(nbytes: int, device) -> torch.Tensor:
 
 
 class CompressedKVCache:
-    """Caller-owned compressed cache: one device buffer carved by tria_cache_init."""
+    """Caller-owned compressed cache: one device buffer carved by tria_cache_init
+    (contiguous [B, Hkv, capacity] rows)."""
 
     def __init__(self, B: int, Hkv: int, D: int, T: int, capacity: int, device="cuda"):
         n = lib().tria_cache_bytes(B, Hkv, D, T, capacity)
         if n == 0:
             raise TriaError("tria_cache_bytes", TRIA_ERR_INVALID_ARG)
         self.buffer = _aligned_empty(n, device)
+        self.buffer[:256].zero_()                  # the status word
         self.struct = tria_kv_cache()
         _check("tria_cache_init", lib().tria_cache_init(ctypes.byref(self.struct), _dev_ptr(self.buffer), n,
                                                          B, Hkv, D, T, capacity))
         self.B, self.Hkv, self.D, self.T, self.capacity = B, Hkv, D, T, capacity
+        self.lead = (B, Hkv, capacity)
 
     def plane(self, name: str) -> torch.Tensor:
-        """View of one plane: k8/v8 int8 [B,Hkv,cap,D], k4/v4 uint8 [B,Hkv,cap,D/2], *_scale fp32 [B,Hkv,cap]."""
+        """View of one plane: k8/v8 int8 [*lead, D], k4/v4 uint8 [*lead, D/2], *_scale fp32 [*lead]
+        (lead = (B, Hkv, capacity) contiguous, (num_pages, Hkv, T) paged)."""
         base = self.buffer.data_ptr()
         off = getattr(self.struct, name) - base
-        rows = self.B * self.Hkv * self.capacity
+        rows = int(np.prod(self.lead))
         if name in ("k8", "v8"):
-            return self.buffer[off:off + rows * self.D].view(torch.int8).view(self.B, self.Hkv, self.capacity, self.D)
+            return self.buffer[off:off + rows * self.D].view(torch.int8).view(*self.lead, self.D)
         if name in ("k4", "v4"):
-            return self.buffer[off:off + rows * self.D // 2].view(self.B, self.Hkv, self.capacity, self.D // 2)
-        return self.buffer[off:off + rows * 4].view(torch.float32).view(self.B, self.Hkv, self.capacity)
+            return self.buffer[off:off + rows * self.D // 2].view(*self.lead, self.D // 2)
+        return self.buffer[off:off + rows * 4].view(torch.float32).view(*self.lead)
+
+    def status(self, stream=None) -> int:
+        """The cache's device error word (synchronises; clears it)."""
+        return int(lib().tria_cache_status(ctypes.byref(self.struct), _stream(stream)))
+
+
+class PagedKVCache(CompressedKVCache):
+    """Caller-owned paged compressed cache: a pool of `num_pages` pages of T tokens x Hkv
+    heads carved by tria_paged_cache_init, addressed through `block_table` (a device int32
+    tensor [B, max_blocks] of page ids that the caller owns and may update between calls)."""
+
+    def __init__(self, B: int, Hkv: int, D: int, T: int, num_pages: int, block_table: torch.Tensor,
+                 device="cuda"):
+        n = lib().tria_paged_cache_bytes(num_pages, Hkv, D, T)
+        if n == 0:
+            raise TriaError("tria_paged_cache_bytes", TRIA_ERR_INVALID_ARG)
+        if block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != B:
+            raise ValueError("block_table must be a device int32 tensor [B, max_blocks]")
+        self.block_table = block_table
+        self.buffer = _aligned_empty(n, device)
+        self.buffer[:256].zero_()
+        self.struct = tria_kv_cache()
+        mb = block_table.shape[1]
+        _check("tria_paged_cache_init", lib().tria_paged_cache_init(
+            ctypes.byref(self.struct), _dev_ptr(self.buffer), n, B, Hkv, D, T, num_pages, _dev_ptr(block_table), mb))
+        self.B, self.Hkv, self.D, self.T, self.capacity = B, Hkv, D, T, mb * T
+        self.num_pages, self.max_blocks = num_pages, mb
+        self.lead = (num_pages, Hkv, T)
 
 
 def tria_quantize_rows(X: torch.Tensor, int4: bool = True, stream=None):
@@ -281,3 +320,71 @@ def tria_decode_static(q: torch.Tensor, cache: CompressedKVCache, kv_len, hi, ke
         hi_a.ctypes.data_as(ctypes.c_void_p), keep_a.ctypes.data_as(ctypes.c_void_p), _dev_ptr(O), _dev_ptr(LSE),
         _stream(stream)))
     return O, LSE
+
+
+def tria_decode_static_status(stream=None) -> int:
+    """Error word of the fixed scratch tria_decode_static uses in the current context (synchronises)."""
+    L = lib()
+    if not getattr(L.tria_decode_static_status, "_typed", False):
+        L.tria_decode_static_status.argtypes = [ctypes.c_void_p]
+        L.tria_decode_static_status.restype = ctypes.c_int
+        L.tria_decode_static_status._typed = True
+    return int(L.tria_decode_static_status(_stream(stream)))
+
+
+# ---------------------------------------------------------------- calibration
+
+def _typed(name, argtypes, restype):
+    f = getattr(lib(), name)
+    if not getattr(f, "_typed", False):
+        f.argtypes, f.restype, f._typed = argtypes, restype, True
+    return f
+
+
+def tria_calibration_costs(nb: int, T: int, D: int, cand_hi, cand_keep) -> np.ndarray:
+    """Cost of each candidate (hi, keep) for one head over nb x nb causal blocks (int64 [C])."""
+    P = ctypes.c_void_p
+    f = _typed("tria_calibration_costs", [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, ctypes.c_int, P],
+               ctypes.c_int)
+    h, k = _host_i32(cand_hi), _host_i32(cand_keep)
+    out = np.zeros(len(h), np.int64)
+    _check("tria_calibration_costs", f(nb, T, D, h.ctypes.data_as(P), k.ctypes.data_as(P), len(h),
+                                       out.ctypes.data_as(P)))
+    return out
+
+
+def tria_calibrate(Q: torch.Tensor, cache: CompressedKVCache, W_O: torch.Tensor, cand_hi, cand_keep,
+                   workspace: torch.Tensor | None = None, stream=None):
+    """Per-candidate, per-head error after the output projection and per-head energy
+    (float64 numpy [C, Hq] and [Hq]); the normalised error is err / energy.sum()."""
+    P, I = ctypes.c_void_p, ctypes.c_int
+    B, Hq, S, D = Q.shape
+    dims = tria_dims(B, Hq, cache.Hkv, S, D, cache.T)
+    d_model = W_O.shape[1]
+    need = _typed("tria_calibrate_workspace_bytes", [ctypes.POINTER(tria_dims), I], ctypes.c_size_t)(
+        ctypes.byref(dims), d_model)
+    if need == 0:
+        raise TriaError("tria_calibrate_workspace_bytes", TRIA_ERR_INVALID_ARG)
+    if workspace is None:
+        workspace = _aligned_empty(need, Q.device)
+    h, k = _host_i32(cand_hi), _host_i32(cand_keep)
+    err = np.zeros((len(h), Hq), np.float64)
+    energy = np.zeros(Hq, np.float64)
+    f = _typed("tria_calibrate", [P, ctypes.POINTER(tria_kv_cache), ctypes.POINTER(tria_dims), P, I, P, P, I, P, P,
+                                  P, ctypes.c_size_t, P], I)
+    _check("tria_calibrate", f(_dev_ptr(Q), ctypes.byref(cache.struct), ctypes.byref(dims), _dev_ptr(W_O), d_model,
+                               h.ctypes.data_as(P), k.ctypes.data_as(P), len(h), err.ctypes.data_as(P),
+                               energy.ctypes.data_as(P), _dev_ptr(workspace), workspace.numel(), _stream(stream)))
+    return err, energy
+
+
+def tria_allocate(err, cost, budget: int) -> np.ndarray:
+    """Greedy global allocation: err [C, H] float64, cost [C, H] int64 -> chosen candidate per head."""
+    P = ctypes.c_void_p
+    f = _typed("tria_allocate", [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int64, P], ctypes.c_int)
+    e = np.ascontiguousarray(err, np.float64)
+    c = np.ascontiguousarray(cost, np.int64)
+    C, H = e.shape
+    out = np.zeros(H, np.int32)
+    _check("tria_allocate", f(e.ctypes.data_as(P), c.ctypes.data_as(P), C, H, int(budget), out.ctypes.data_as(P)))
+    return out

@@ -58,7 +58,7 @@ typedef enum {
 } tria_status;
 
 /* Compressed KV cache: the "prepared K and V" of the method, one row per token.
- * For X in {k, v}:
+ * For X in {k, v}, in the contiguous layout (block_table == NULL):
  *   x8        int8  [B, Hkv, capacity, D]      8-bit codes
  *   x4        uint8 [B, Hkv, capacity, D/2]    4-bit codes, two per byte:
  *                                              element 2m in the low nibble,
@@ -66,8 +66,20 @@ typedef enum {
  *                                              4-bit two's complement
  *   x8_scale  fp32  [B, Hkv, capacity]         per-token scale of the 8-bit plane
  *   x4_scale  fp32  [B, Hkv, capacity]         per-token scale of the 4-bit plane
- * All eight pointers are device pointers, 16-byte aligned. capacity is a
- * multiple of T. The struct itself is host memory, read during the call only. */
+ * In the paged layout (block_table != NULL) the planes are a pool of num_pages
+ * pages of T tokens of every KV head -- x8 [num_pages, Hkv, T, D], x4
+ * [num_pages, Hkv, T, D/2], scales [num_pages, Hkv, T] -- and logical block j
+ * (tokens [jT, jT + T)) of sequence b lives in page block_table[b * max_blocks
+ * + j]; capacity = max_blocks * T tokens per sequence. block_table is a device
+ * int32 array the caller owns and may change between calls (pages handed out
+ * as a sequence grows). Pages written by one call must not be shared by two
+ * sequences.
+ * status is a device int, the cache's error word: a page id outside
+ * [0, num_pages) met by any kernel sets TRIA_ERR_BOUNDS there and that access is
+ * skipped (reads go to page 0 instead); tria_cache_status reads and clears it.
+ * All pointers are device pointers, the planes 16-byte aligned; capacity is a
+ * multiple of T. The struct itself is host memory, read during the call only.
+ * tria_cache_init / tria_paged_cache_init fill it. */
 typedef struct {
   int8_t* k8;
   uint8_t* k4;
@@ -78,6 +90,9 @@ typedef struct {
   float* v8_scale;
   float* v4_scale;
   int B, Hkv, D, T, capacity;
+  const int32_t* block_table;   /* NULL: contiguous; else device int32 [B, max_blocks] */
+  int max_blocks, num_pages;    /* paged layout only */
+  int* status;                  /* device error word */
 } tria_kv_cache;
 
 /* Shape of a prefill: B sequences of S tokens, Hq query heads, Hkv KV heads. */
@@ -88,16 +103,40 @@ typedef struct {
 /* Human-readable name of a status code (static string). */
 const char* tria_status_string(int status);
 
-/* Bytes needed to hold every plane of a cache carved by tria_cache_init. */
+/* Bytes needed to hold every plane and the status word of a contiguous cache
+ * carved by tria_cache_init. */
 size_t tria_cache_bytes(int B, int Hkv, int D, int T, int capacity);
 
 /* Fill `cache` with plane pointers carved from one caller buffer `base`
- * (device, 256-byte aligned, at least tria_cache_bytes(...) bytes). Writes no
- * device memory. Returns TRIA_ERR_INVALID_ARG on a bad shape or alignment. */
+ * (device, 256-byte aligned, at least tria_cache_bytes(...) bytes), contiguous
+ * layout. Writes no device memory: the caller zeroes the buffer (or calls
+ * tria_cache_status once) before the status word is read. Returns
+ * TRIA_ERR_INVALID_ARG on a bad shape or alignment. */
 int tria_cache_init(tria_kv_cache* cache, void* base, size_t bytes,
                     int B, int Hkv, int D, int T, int capacity);
 
+/* Paged compressed cache (the "special KV-cache layout" the rit.work TriAttention
+ * page, section "Когда TriAttention меняет планы инфраструктуры", paragraph four,
+ * says a deployment must support; pages of T tokens named by a block table, as
+ * paged KV caches do). Bytes of a pool of num_pages pages plus the status word. */
+size_t tria_paged_cache_bytes(int num_pages, int Hkv, int D, int T);
+
+/* Fill `cache` for a paged pool carved from `base` (device, 256-byte aligned,
+ * at least tria_paged_cache_bytes(...) bytes) serving B sequences through
+ * `block_table` (device int32 [B, max_blocks], caller-owned, read by every call
+ * that uses the cache). Writes no device memory. Returns TRIA_ERR_INVALID_ARG
+ * on a bad shape, alignment or NULL table. */
+int tria_paged_cache_init(tria_kv_cache* cache, void* base, size_t bytes, int B, int Hkv, int D, int T,
+                          int num_pages, const int32_t* block_table, int max_blocks);
+
+/* Synchronise `stream`, return the cache's status word (TRIA_OK or
+ * TRIA_ERR_BOUNDS after a page id out of range) and clear it. */
+int tria_cache_status(const tria_kv_cache* cache, void* stream);
+
 /* Codec over arbitrary rows (used for Q and by the tests).
+ * Passage: rit.work TriAttention page, section "Какие связи можно не считать, а
+ * какие нельзя удалять", paragraph three (blocks computed at 8 or at 4 bits);
+ * the per-token symmetric rule above is a reading of it.
  * X: device bf16 [rows, D]. Outputs (device): c8 int8 [rows, D], s8 fp32
  * [rows], c4 uint8 [rows, D/2] packed as in the cache, s4 fp32 [rows].
  * Any of c4/s4 may be NULL to skip that plane. Bit-exact with the codec rule
@@ -106,9 +145,16 @@ int tria_quantize_rows(const void* X, int64_t rows, int D, int8_t* c8, float* s8
                        uint8_t* c4, float* s4, void* stream);
 
 /* Write the prepared K/V of S tokens into cache positions [start, start+S).
+ * Passage: rit.work TriAttention page, section "Как калибровка распределяет
+ * вычисления между головами", last paragraph -- the prepared keys and values go
+ * into a compressed KV cache that step-by-step generation reads; the 8-bit and
+ * 4-bit planes are the two precisions of section "Какие связи можно не считать, а
+ * какие нельзя удалять", paragraph three. Both planes of every token are written,
+ * because the plane a tile uses depends on the query block that reads it.
  * K, V: device bf16 [B, Hkv, S, D] (B, Hkv, D as in the cache).
  * Requires 0 <= start, start + S <= capacity, S >= 1. Any start is allowed, so
- * this also appends decode tokens one at a time (S = 1). */
+ * this also appends decode tokens one at a time (S = 1). Errors: INVALID_ARG on
+ * a bad range or pointer, UNSUPPORTED off sm_100a; nothing is written then. */
 int tria_quantize_kv(const void* K, const void* V, int S, int start,
                      const tria_kv_cache* cache, void* stream);
 
@@ -134,6 +180,13 @@ int tria_prefill_load_plan(int nb, int T, int hi, int keep, int32_t* plan, int64
 size_t tria_prefill_workspace_bytes(const tria_dims* dims);
 
 /* Fused block-sparse mixed-precision causal prefill.
+ * Passage: rit.work TriAttention page, section "Какие связи можно не считать, а
+ * какие нельзя удалять", paragraphs three to five (per tile: skip, 4 bits or
+ * 8 bits, from the distance to the diagonal and the head's two boundaries; key
+ * block 0 and the diagonal always at 8 bits), and section "Как калибровка
+ * распределяет вычисления между головами", last paragraph (one fused kernel
+ * takes the kept blocks grouped by precision and reduces them into one
+ * normalised result).
  * Q: device bf16 [B, Hq, S, D]; cache: holds K/V tokens [0, S) (written by
  * tria_quantize_kv); hi, keep: HOST int32 arrays of length Hq with
  * 0 <= hi <= keep (keep may exceed the block count). S % T == 0,
@@ -162,6 +215,11 @@ int tria_prefill_attend(const tria_kv_cache* cache, const tria_dims* dims, const
 size_t tria_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int T, int capacity);
 
 /* Split-KV decode of one new token per sequence over the compressed cache.
+ * Passage: rit.work TriAttention page, section "Как калибровка распределяет
+ * вычисления между головами", last paragraph (the chosen boundaries are used in
+ * both stages; generation reads the prepared K/V from the compressed cache and so
+ * reads less data), with decode bound by memory traffic (llmis.ru chapter 3.5,
+ * section 2). The new token is one row of the prefill problem.
  * q: device bf16 [B, Hq, D]; kv_len: HOST int32 [B], 1 <= kv_len[b] <=
  * capacity: the token sits at position kv_len[b]-1 and is already in the
  * cache, so its block is the diagonal block. hi, keep: HOST int32 [Hq].
@@ -189,14 +247,66 @@ int tria_decode(const void* q, const tria_kv_cache* cache, const int32_t* kv_len
  * up the array's device address (cudaGetSymbolAddress) with that device
  * current; make that first call before any stream capture. All calls on a
  * device share the array: each call clears what must start at zero, and calls
- * whose GPU work overlaps (unordered streams) race on it. Device-side pipeline
- * errors land in the shared array's error word and are not reported here. */
+ * whose GPU work overlaps (unordered streams) race on it. The address is looked
+ * up per CUDA context, so a context the caller created and made current gets its
+ * own copy of the array. A device-side pipeline error (a wait past its limit)
+ * makes that call's O and LSE NaN and lands in the array's error word, which
+ * tria_decode_static_status reads. */
 int tria_decode_static(const void* q, const tria_kv_cache* cache, const int32_t* kv_len, int Hq,
                        const int32_t* hi, const int32_t* keep, void* O, float* LSE, void* stream);
 
+/* Synchronise `stream` and return the device-side error word of the fixed
+ * scratch array that tria_decode_static uses in the current context (TRIA_OK,
+ * TRIA_ERR_TIMEOUT or TRIA_ERR_BOUNDS); every tria_decode_static call clears it.
+ * No counterpart in the paper. Allocates nothing. */
+int tria_decode_static_status(void* stream);
+
+/* ---- Calibration of the per-head boundaries and the global allocator ----
+ * Passage: rit.work TriAttention page, section "Как калибровка распределяет
+ * вычисления между головами", paragraphs one to three: candidate boundary pairs
+ * are tried for every head; a candidate's error is measured after the output
+ * projection and normalised by the energy of the layer's output; each candidate
+ * has a cost counting whole processed blocks (query-key product, normalisation
+ * of the weights, aggregation of the values); a global allocator adds work where
+ * it lowers the error most. Readings: the reference output keeps every block at
+ * 8 bits; error of head h = sum over its rows of ||(O_c - O_ref) W_O[h]||^2, with
+ * W_O[h] the D rows of W_O that head h feeds; energy of head h = sum over rows of
+ * ||O_ref W_O[h]||^2 (cross terms between heads dropped in both); a kept tile
+ * costs 4 T^2 D + 4 T^2 at 8 bits and 2 T^2 D + 4 T^2 at 4 bits. */
+
+/* Cost of each candidate (cand_hi[c], cand_keep[c]) for one head over nb x nb
+ * causal blocks of T tokens, head dim D: host-only. cost: host int64 [C]. */
+int tria_calibration_costs(int nb, int T, int D, const int32_t* cand_hi, const int32_t* cand_keep, int C,
+                           int64_t* cost);
+
+/* Workspace bytes tria_calibrate needs (0 if the arguments are invalid). */
+size_t tria_calibrate_workspace_bytes(const tria_dims* dims, int d_model);
+
+/* Errors of C candidate boundary pairs, applied to every head at once, on one
+ * layer's calibration sample. Q: device bf16 [B, Hq, S, D]; cache: holds that
+ * sample's K/V (tokens [0, S)); W_O: device bf16 [Hq * D, d_model], row-major
+ * (row h * D + k is what output element k of head h multiplies). cand_hi,
+ * cand_keep: HOST int32 [C]. Writes HOST err [C, Hq] (the unnormalised errors
+ * E[c][h]) and energy [Hq]; the normalised error is E / sum(energy). Runs the
+ * fused prefill once for the reference and once per candidate, then waits for
+ * the stream (the results are host memory). Returns a device-side error word of
+ * the prefill as tria_workspace_status does, else TRIA_OK. */
+int tria_calibrate(const void* Q, const tria_kv_cache* cache, const tria_dims* dims, const void* W_O, int d_model,
+                   const int32_t* cand_hi, const int32_t* cand_keep, int C, double* err, double* energy,
+                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* Greedy global allocation (host-only). err: host double [C, H], cost: host
+ * int64 [C, H]; every head starts at its cheapest candidate (then the lower
+ * error, then the first); then, while the total cost stays within `budget`, the
+ * single move of one head to a costlier candidate with a lower error that has the
+ * largest error decrease per unit of added cost is taken (the first in
+ * head-then-candidate order on equal ratios). choice: host int32 [H]. */
+int tria_allocate(const double* err, const int64_t* cost, int C, int H, int64_t budget, int32_t* choice);
+
 /* Synchronise `stream` and return the device-side error word of `workspace`
  * (TRIA_OK, TRIA_ERR_TIMEOUT or TRIA_ERR_BOUNDS); the word is cleared by
- * every tria_prefill / tria_decode call that uses this workspace. */
+ * every tria_prefill / tria_decode call that uses this workspace. After a
+ * decode whose wait ran past its limit, that call's O and LSE are NaN. */
 int tria_workspace_status(const void* workspace, void* stream);
 
 #ifdef __cplusplus

@@ -16,11 +16,19 @@ def L():
     return tria.lib()
 
 
+EXPECTED = {
+    "tria_status_string", "tria_cache_bytes", "tria_cache_init", "tria_quantize_rows", "tria_quantize_kv",
+    "tria_count_tiles", "tria_prefill_load_plan", "tria_prefill_workspace_bytes", "tria_prefill",
+    "tria_prefill_prepare", "tria_prefill_attend", "tria_decode_workspace_bytes", "tria_decode",
+    "tria_decode_static", "tria_decode_static_status", "tria_workspace_status",
+    "tria_paged_cache_bytes", "tria_paged_cache_init", "tria_cache_status",
+    "tria_calibration_costs", "tria_calibrate_workspace_bytes", "tria_calibrate", "tria_allocate",
+}
+
+
 def test_every_declared_symbol_is_exported(L):
     names = tria.declared_functions()
-    assert len(names) == 15, names
-    for n in ("tria_quantize_kv", "tria_prefill", "tria_decode", "tria_quantize_rows"):
-        assert n in names
+    assert set(names) == EXPECTED, sorted(set(names) ^ EXPECTED)
     for n in names:
         assert hasattr(L, n), f"{n} declared in tria.h but not exported"
 
@@ -42,13 +50,39 @@ def test_cache_sizes_and_carving(L):
     base = 1 << 40                                             # never dereferenced
     assert L.tria_cache_init(ctypes.byref(c), ctypes.c_void_p(base), n, B, Hkv, D, T, cap) == 0
     ptrs = [c.k8, c.k4, c.k8_scale, c.k4_scale, c.v8, c.v4, c.v8_scale, c.v4_scale]
-    assert ptrs[0] == base and all(p % 256 == 0 for p in ptrs)
+    assert c.status == base and ptrs[0] >= base + 4 and all(p % 256 == 0 for p in ptrs)
+    assert c.block_table is None and c.capacity == cap
     sizes = [rows * D, rows * D // 2, rows * 4, rows * 4] * 2
     for p, q, s in zip(ptrs, ptrs[1:], sizes):
         assert q - p >= s                                      # planes do not overlap
     assert ptrs[-1] + rows * 4 <= base + n
     assert L.tria_cache_init(ctypes.byref(c), ctypes.c_void_p(base + 16), n, B, Hkv, D, T, cap) == 1
     assert L.tria_cache_init(ctypes.byref(c), ctypes.c_void_p(base), n - 1, B, Hkv, D, T, cap) == 1
+
+
+def test_paged_cache_sizes_and_carving(L):
+    pages, Hkv, D, T, B, mb = 37, 2, 64, 128, 3, 5
+    n = L.tria_paged_cache_bytes(pages, Hkv, D, T)
+    rows = pages * Hkv * T
+    assert n >= 4 + 2 * (rows * D + rows * D // 2 + 2 * rows * 4)
+    assert L.tria_paged_cache_bytes(0, Hkv, D, T) == 0
+    assert L.tria_paged_cache_bytes(pages, Hkv, D, 96) == 0
+    c = tria.tria_kv_cache()
+    base, table = 1 << 40, 1 << 41                             # never dereferenced
+    assert L.tria_paged_cache_init(ctypes.byref(c), ctypes.c_void_p(base), n, B, Hkv, D, T, pages,
+                                   ctypes.c_void_p(table), mb) == 0
+    assert c.block_table == table and c.max_blocks == mb and c.num_pages == pages and c.capacity == mb * T
+    ptrs = [c.k8, c.k4, c.k8_scale, c.k4_scale, c.v8, c.v4, c.v8_scale, c.v4_scale]
+    sizes = [rows * D, rows * D // 2, rows * 4, rows * 4] * 2
+    for p, q, sz in zip(ptrs, ptrs[1:], sizes):
+        assert q - p >= sz
+    assert ptrs[-1] + rows * 4 <= base + n
+    # no table, a short buffer, a misaligned base
+    assert L.tria_paged_cache_init(ctypes.byref(c), ctypes.c_void_p(base), n, B, Hkv, D, T, pages, None, mb) == 1
+    assert L.tria_paged_cache_init(ctypes.byref(c), ctypes.c_void_p(base), n - 1, B, Hkv, D, T, pages,
+                                   ctypes.c_void_p(table), mb) == 1
+    assert L.tria_paged_cache_init(ctypes.byref(c), ctypes.c_void_p(base + 16), n, B, Hkv, D, T, pages,
+                                   ctypes.c_void_p(table), mb) == 1
 
 
 def test_tile_counts_match_oracle(L, oracle_mod):
@@ -115,3 +149,31 @@ def test_host_validation_rejects_bad_arguments(L):
     assert L.tria_quantize_rows(fake, 4, 96, fake, fake, fake, fake, None) == tria.TRIA_ERR_UNSUPPORTED
     assert L.tria_quantize_rows(ctypes.c_void_p((1 << 41) + 2), 4, 128, fake, fake, fake, fake,
                                 None) == tria.TRIA_ERR_INVALID_ARG
+
+
+def test_calibration_costs_match_oracle(L):
+    from oracle import calibration as cal
+    for nb, T, D in ((8, 64, 128), (37, 128, 64), (1, 64, 64)):
+        hi = [0, 1, 2, 5, nb, 3]
+        keep = [0, 3, 2, 9, nb, 40]
+        assert tria.tria_calibration_costs(nb, T, D, hi, keep).tolist() == \
+            cal.candidate_costs(nb, T, D, hi, keep).tolist()
+    with pytest.raises(tria.TriaError):
+        tria.tria_calibration_costs(8, 64, 128, [3], [2])
+
+
+def test_allocator_matches_oracle(L):
+    """The library's greedy allocator takes the same decisions as the oracle's on the same
+    (error, cost) tables: the hand-worked example and random tables with ties."""
+    from oracle import calibration as cal
+    err = np.array([[9.0, 4.0, 6.0], [3.0, 3.0, 5.0], [1.0, 0.0, 0.5]])
+    cost = np.array([[10, 10, 10], [20, 20, 20], [40, 40, 40]], np.int64)
+    for budget in (30, 45, 80, 1000):
+        assert tria.tria_allocate(err, cost, budget).tolist() == cal.allocate(err, cost, budget)
+    rng = np.random.RandomState(7)
+    for _ in range(300):
+        C, H = rng.randint(1, 7), rng.randint(1, 9)
+        cost = rng.randint(1, 12, (C, H)).astype(np.int64)          # small ranges: many ties
+        err = rng.randint(0, 6, (C, H)).astype(np.float64) / 4.0
+        budget = int(rng.randint(0, 80))
+        assert tria.tria_allocate(err, cost, budget).tolist() == cal.allocate(err, cost, budget)

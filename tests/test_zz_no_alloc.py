@@ -60,14 +60,25 @@ def test_static_scratch_decode_matches_workspace_decode():
         compare_o(O, O_ref.double().cpu().numpy(), "static scratch decode")
         compare_lse(LSE, L_ref.double().cpu().numpy(), "static scratch decode")
 
-    # a problem whose decode scratch exceeds the fixed array is refused before any work
-    big = tria.tria_kv_cache()
-    n = L.tria_cache_bytes(1024, 2, 128, 128, 128)
-    assert L.tria_cache_init(ctypes.byref(big), ctypes.c_void_p(1 << 40), n, 1024, 2, 128, 128, 128) == 0
-    assert tria.tria_decode_workspace_bytes(1024, 32, 2, 128, 128, 128) > (40 << 20)
-    kv = host([128] * 1024)
-    h = host([1] * 32)
-    dummy = ctypes.c_void_p(1 << 41)
-    st = L.tria_decode_static(dummy, ctypes.byref(big), kv.ctypes.data_as(P), 32, h.ctypes.data_as(P),
-                              h.ctypes.data_as(P), dummy, dummy, stream)
+        # the fixed array's error word: clear after a call that completed normally
+        L.tria_decode_static_status.argtypes = [P]
+        L.tria_decode_static_status.restype = ctypes.c_int
+        assert L.tria_decode_static_status(stream) == tria.TRIA_OK
+
+    # A problem whose decode scratch exceeds the fixed array is refused before any
+    # work. Its buffers are real allocations of the right sizes, so that a
+    # regression in the size check would give a wrong status, never a launch on
+    # made-up addresses.
+    Bb, Hqb, Hkvb, Db, Tb, capb = 1024, 32, 2, 128, 128, 128
+    assert tria.tria_decode_workspace_bytes(Bb, Hqb, Hkvb, Db, Tb, capb) > (40 << 20)
+    big = tria.CompressedKVCache(Bb, Hkvb, Db, Tb, capb)
+    qb = torch.zeros((Bb, Hqb, Db), dtype=torch.bfloat16, device="cuda")
+    Ob = torch.zeros_like(qb)
+    Lb = torch.zeros((Bb, Hqb), dtype=torch.float32, device="cuda")
+    kv = host([capb] * Bb)
+    h = host([1] * Hqb)
+    st = L.tria_decode_static(ptr(qb), ctypes.byref(big.struct), kv.ctypes.data_as(P), Hqb, h.ctypes.data_as(P),
+                              h.ctypes.data_as(P), ptr(Ob), ptr(Lb), stream)
     assert st == tria.TRIA_ERR_WORKSPACE
+    torch.cuda.synchronize()
+    assert int(Ob.view(torch.int16).abs().sum()) == 0 and float(Lb.abs().sum()) == 0.0   # nothing written
