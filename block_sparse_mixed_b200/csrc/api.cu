@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -20,6 +21,9 @@ namespace tria {
 namespace {
 
 constexpr int kRowsPerTile = 128;   // query rows of a fused-prefill tile
+
+// Whether the fused prefill may use the GQA-shared kernel (tria_prefill_gqa).
+std::atomic<bool> g_prefill_gqa{true};
 
 constexpr size_t kAlign = 256;
 
@@ -141,7 +145,7 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? TRIA_OK : TRIA_ERR_CU
 // ---------------------------------------------------------------- workspace layouts
 
 struct PrefillLayout {
-  size_t ctrl, q8, q4, q8s, q4s, k4x, k8x, vd8, vd4, total;
+  size_t ctrl, q8, q4, q8s, q4s, k4x, k8x, vt8, vt4, total;
 };
 
 PrefillLayout prefill_layout(const tria_dims& d) {
@@ -156,8 +160,8 @@ PrefillLayout prefill_layout(const tria_dims& d) {
   L.q4s = off; off += align_up(qrows * 4);
   L.k4x = off; off += align_up(krows * kQKRowBytes);
   L.k8x = off; if (d.D < 128) off += align_up(krows * kQKRowBytes);
-  L.vd8 = off; off += align_up(krows * d.D * 2);
-  L.vd4 = off; off += align_up(krows * d.D * 2);
+  L.vt8 = off; off += align_up(krows * d.D * 2);
+  L.vt4 = off; off += align_up(krows * d.D * 2);
   L.total = off;
   return L;
 }
@@ -367,6 +371,11 @@ int tria_prefill_load_plan(int nb, int T, int hi, int keep, int32_t* plan, int64
   return TRIA_OK;
 }
 
+int tria_prefill_gqa(int enable) {
+  const bool was = g_prefill_gqa.exchange(enable != 0);
+  return was ? 1 : 0;
+}
+
 size_t tria_prefill_workspace_bytes(const tria_dims* dims) {
   if (check_dims(dims) != TRIA_OK) return 0;
   return prefill_layout(*dims).total;
@@ -423,10 +432,10 @@ int tria_prefill_prepare(const void* Q, const tria_kv_cache* cache, const tria_d
   pa.v8s = cache->v8_scale; pa.v4s = cache->v4_scale;
   pa.k8x = d.D < 128 ? reinterpret_cast<int8_t*>(ws + L.k8x) : nullptr;
   pa.k4x = reinterpret_cast<int8_t*>(ws + L.k4x);
-  pa.vd8 = reinterpret_cast<__nv_bfloat16*>(ws + L.vd8);
-  pa.vd4 = reinterpret_cast<__nv_bfloat16*>(ws + L.vd4);
-  pa.ci = cache_index(*cache); pa.S = d.S; pa.groups = groups;
-  if (launch_prepare(pa, d.D, st) != cudaSuccess) return TRIA_ERR_CUDA;
+  pa.vt8 = reinterpret_cast<__nv_bfloat16*>(ws + L.vt8);
+  pa.vt4 = reinterpret_cast<__nv_bfloat16*>(ws + L.vt4);
+  pa.ci = cache_index(*cache); pa.S = d.S; pa.nb = nb; pa.groups = groups;
+  if (launch_prepare(pa, d.D, d.T, st) != cudaSuccess) return TRIA_ERR_CUDA;
   return TRIA_OK;
 }
 
@@ -450,8 +459,10 @@ int tria_prefill_attend(const tria_kv_cache* cache, const tria_dims* dims, const
   bool ok = make_map(&maps.q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + L.q8, kQKRowBytes, qrows, 128, 128) &&
             make_map(&maps.q4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + L.q4, kQKRowBytes, qrows, 128, 128) &&
             make_map(&maps.k4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + L.k4x, kQKRowBytes, krows, 128, d.T) &&
-            make_map(&maps.v8, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + L.vd8, d.D, krows, 64, d.T) &&
-            make_map(&maps.v4, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + L.vd4, d.D, krows, 64, d.T);
+            make_map(&maps.v8, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + L.vt8, d.T,
+                     static_cast<uint64_t>(groups) * nb * d.D, 64, d.D) &&
+            make_map(&maps.v4, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ws + L.vt4, d.T,
+                     static_cast<uint64_t>(groups) * nb * d.D, 64, d.D);
   const CacheIndex ci = cache_index(*cache);
   if (d.D == 128)
     ok = ok && make_map(&maps.k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, cache->k8, 128,
@@ -465,6 +476,11 @@ int tria_prefill_attend(const tria_kv_cache* cache, const tria_dims* dims, const
   a.ci = ci; a.k8_in_cache = d.D == 128;
   a.n_qtiles = (d.S + 127) / 128;
   a.n_units = d.B * d.Hq * a.n_qtiles;
+  // Two query heads of a KV group share one CTA (and every K/V load) when their
+  // boundaries coincide, for every such pair of the launch.
+  bool gqa = g_prefill_gqa.load() && (a.G % 2 == 0);
+  for (int h = 0; gqa && h < d.Hq; h += 2) gqa = hi[h] == hi[h + 1] && keep[h] == keep[h + 1];
+  if (gqa) a.n_units = d.B * d.Hkv * (a.G / 2) * a.n_qtiles;
   a.qk_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d.D)));
   a.q8s = reinterpret_cast<const float*>(ws + L.q8s);
   a.q4s = reinterpret_cast<const float*>(ws + L.q4s);
@@ -474,7 +490,8 @@ int tria_prefill_attend(const tria_kv_cache* cache, const tria_dims* dims, const
   a.work = reinterpret_cast<int*>(ws + L.ctrl) + 4;
   for (int h = 0; h < d.Hq; ++h) { a.hi[h] = hi[h]; a.keep[h] = keep[h]; }
   if (cudaMemsetAsync(a.work, 0, sizeof(int), st) != cudaSuccess) return TRIA_ERR_CUDA;   // tile counter
-  return cuda_status(launch_prefill(a, maps, d.D, d.T, dev.sms, st));
+  return cuda_status(gqa ? launch_prefill_gqa(a, maps, d.D, d.T, dev.sms, st)
+                         : launch_prefill(a, maps, d.D, d.T, dev.sms, st));
 }
 
 int tria_prefill(const void* Q, const tria_kv_cache* cache, const tria_dims* dims, const int32_t* hi,

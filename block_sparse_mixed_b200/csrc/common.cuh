@@ -310,21 +310,6 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
   return d;
 }
 
-// Shared-memory matrix descriptor of an N-major (MN-major) operand tile with the
-// 128-byte swizzle: rows along K of 128 bytes (64 bf16 along N), 8-row groups
-// 1024 bytes apart, and the next 64 values along N `lbo_bytes` further on -- the
-// layout of TMA boxes of 128-byte rows written with CU_TENSOR_MAP_SWIZZLE_128B,
-// one box per 64 values of N. Moving along K by 8 rows adds 1024 bytes.
-__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t smem_addr, uint32_t lbo_bytes) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);   // start address (16-byte units)
-  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;   // leading byte offset: next 64 along N
-  d |= static_cast<uint64_t>(1024 >> 4) << 32;                 // stride byte offset: next 8 rows along K
-  d |= static_cast<uint64_t>(1) << 46;                         // descriptor version (sm_100)
-  d |= static_cast<uint64_t>(2) << 61;                         // layout: 128-byte swizzle
-  return d;
-}
-
 // Instruction descriptors (kind::i8 int8 x int8 -> s32; kind::f16 bf16 x bf16 -> f32),
 // both operands K-major, dense.
 __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
@@ -339,8 +324,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
-// kind::f16 bf16 x bf16 -> f32 with A K-major and B N-major (bit 16: B transposed).
-__host__ __device__ constexpr uint32_t idesc_bf16_bn(int M, int N) { return idesc_bf16(M, N) | (1u << 16); }
 
 // Hardware base-2 exponential (MUFU ex2, approximate, flushes subnormal results to 0).
 __device__ __forceinline__ float fast_exp2(float x) {

@@ -70,10 +70,11 @@ struct PrepareArgs {
   const float* v4s;
   int8_t* k8x;        // null when D == 128 (the cache plane is read directly)
   int8_t* k4x;        // [groups * S, 128]
-  __nv_bfloat16* vd8; // [groups * S, D] V of the 8-bit plane, dequantised
-  __nv_bfloat16* vd4; // [groups * S, D] V of the 4-bit plane, dequantised
+  __nv_bfloat16* vt8; // [groups * nb, D, T] V of the 8-bit plane, dequantised, transposed per block
+  __nv_bfloat16* vt4; // [groups * nb, D, T] the same for the 4-bit plane
   CacheIndex ci;
   int64_t S;          // prefill tokens per (b, kv head) (= nb * T)
+  int64_t nb;
   int64_t groups;     // B * Hkv
 };
 
@@ -130,9 +131,11 @@ struct DecodeArgs {
 };
 
 cudaError_t launch_quant_rows(const QuantArgs& a, int D, cudaStream_t stream);
-cudaError_t launch_prepare(const PrepareArgs& a, int D, cudaStream_t stream);
+cudaError_t launch_prepare(const PrepareArgs& a, int D, int T, cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillArgs& a, const PrefillMaps& maps, int D, int T, int num_sms,
                            cudaStream_t stream);
+cudaError_t launch_prefill_gqa(const PrefillArgs& a, const PrefillMaps& maps, int D, int T, int num_sms,
+                               cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, const DecodeMaps& maps, int num_sms, cudaStream_t stream);
 
 }  // namespace tria

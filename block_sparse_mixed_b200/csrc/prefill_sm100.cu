@@ -30,10 +30,9 @@
 //               as the pair has read S into registers, so the next S of a pair is
 //               computed while the pair still works on the current one.
 //   warp 18     producer of the V tiles (a ring of 2 stages, one per pair).
-//   warp 19     P.V issuer: O += P.V on kind::f16, bf16 P (K-major) and V (N-major,
-//               the dequantised rows as they lie in memory) from shared memory, fp32 O
-//               in TMEM; each P.V frees its V stage, P buffer and the accumulator for
-//               the pair's next load.
+//   warp 19     P.V issuer: O += P.V on kind::f16, bf16 P and V^T from shared memory,
+//               both K-major, fp32 O in TMEM; each P.V frees its V stage, P buffer and
+//               the accumulator for the pair's next load.
 // Each ring is released as soon as its contents are used (K by the QK's
 // completion, the scales after the softmax's first pass, V and P by the P.V's
 // completion), so no stage is held across another role's round trip.
@@ -51,9 +50,12 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "load_plan.cuh"
+#include "prefill_common.cuh"
 
 namespace tria {
 namespace {
+
+using namespace pf;
 
 constexpr int kRows = 128;              // query rows per tile (tcgen05 M)
 constexpr int kThreads = 640;           // 20 warps
@@ -87,8 +89,8 @@ struct Cfg {
   static constexpr int kBlocksPerLoad = kKeys / T;           // key blocks per load
   static constexpr int kQTile = kRows * kQKRowBytes;         // Q codes of one plane
   static constexpr int kKTile = kKeys * kQKRowBytes;         // K codes of one load
-  static constexpr int kVChunk = kKeys * 128;                // V of one load, 64 values of d: 128 key rows x 128 B
-  static constexpr int kVTile = D * kKeys * 2;               // V of one load: D / 64 chunks
+  static constexpr int kVSub = D * 128;                      // one V sub-tile: D rows x 64 keys
+  static constexpr int kVTile = D * kKeys * 2;               // both V sub-tiles of a load
   static constexpr int kPSub = kRows * 128;                  // one P sub-tile: 128 rows x 64 keys
   static constexpr int kPTile = kRows * kKeys * 2;           // P of one load (bf16)
   static constexpr int kScTile = kKeys * 4;                  // K scales of one load
@@ -114,11 +116,11 @@ struct Cfg {
   static constexpr int kSmem = kSmemNeed > 120 * 1024 ? kSmemNeed : 120 * 1024;
   static_assert(kSmemNeed <= 227 * 1024, "shared memory");
   static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0 && kKTile % 1024 == 0 &&
-                    kVChunk % 1024 == 0 && kPSub % 1024 == 0,
+                    kVSub % 1024 == 0 && kPSub % 1024 == 0,
                 "swizzled operand tiles start on 1024-byte boundaries");
   static constexpr uint32_t kIdescQK = idesc_i8(kRows, kKeys);       // 8-bit plane: int8, int32 S
   static constexpr uint32_t kIdescQK4 = idesc_e4m3(kRows, kKeys);    // 4-bit plane: e4m3, fp32 S (exact)
-  static constexpr uint32_t kIdescPV = idesc_bf16_bn(kRows, D);     // P K-major, V N-major
+  static constexpr uint32_t kIdescPV = idesc_bf16(kRows, D);
 };
 
 constexpr int kUnitRing = 16;           // tiles published ahead of the consumers
@@ -165,106 +167,6 @@ __device__ __forceinline__ Unit unit_of(const PrefillArgs& a, int w, int nqb) {
   u.i0 = qt * nqb;
   u.nq = min(nqb, a.nb - u.i0);
   return u;
-}
-
-// Bounded wait that ignores the abort flag: used on the way out to let copies and
-// tensor-core ops already in flight land before the CTA releases its memory.
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-  const unsigned long long t0 = global_timer();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_timer() - t0 > kWaitLimitNs) return;
-  }
-}
-
-// ---- packed fp32x2 arithmetic (two scores per instruction) ----
-__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void up2(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ float max3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-__device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-
-// Softmax pass 1 over N keys of a row: y = float(acc) * s_k as packed pairs, and
-// the maximum over the visible keys (n <= kmax when MASK).
-// FP: S holds fp32 (the 4-bit plane's e4m3 product, an exact integer) instead of int32.
-template <int N, bool MASK, bool FP>
-__device__ __forceinline__ float scores_and_max(const uint32_t (&r)[N], uint64_t (&y)[N / 2], const float* sk,
-                                                int kmax) {
-  auto cv = [](uint32_t v) { return FP ? __uint_as_float(v) : __int2float_rn(static_cast<int>(v)); };
-  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-  for (int q = 0; q < N / 4; ++q) {
-    const float4 s4 = *reinterpret_cast<const float4*>(sk + 4 * q);
-    const uint64_t u01 = pk2(cv(r[4 * q]), cv(r[4 * q + 1]));
-    const uint64_t u23 = pk2(cv(r[4 * q + 2]), cv(r[4 * q + 3]));
-    y[2 * q] = mul2(u01, pk2(s4.x, s4.y));
-    y[2 * q + 1] = mul2(u23, pk2(s4.z, s4.w));
-    float v0, v1, v2, v3;
-    up2(y[2 * q], v0, v1);
-    up2(y[2 * q + 1], v2, v3);
-    if (MASK) {
-      const int n = 4 * q;
-      v0 = n <= kmax ? v0 : -INFINITY;
-      v1 = n + 1 <= kmax ? v1 : -INFINITY;
-      v2 = n + 2 <= kmax ? v2 : -INFINITY;
-      v3 = n + 3 <= kmax ? v3 : -INFINITY;
-    }
-    mx[(q % 2) * 2] = max3(mx[(q % 2) * 2], v0, v1);
-    mx[(q % 2) * 2 + 1] = max3(mx[(q % 2) * 2 + 1], v2, v3);
-  }
-  return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-}
-
-// Softmax pass 2 over N keys: p = 2^(y * alpha - m) as bf16 pairs, stored as they
-// are made into the thread's 128-byte P row (16-byte chunk c at c ^ swz), their
-// fp32 sum accumulated in `acc`; masked keys (n > kmax when MASK) give 0.
-template <int N, bool MASK>
-__device__ __forceinline__ void probs(const uint64_t (&y)[N / 2], uint64_t al2, uint64_t nm2, int kmax,
-                                      uint8_t* prow, int swz, uint64_t (&acc)[4]) {
-#pragma unroll
-  for (int c = 0; c < N / 8; ++c) {
-    uint32_t w[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int k = 4 * c + e;
-      float t0, t1;
-      up2(fma2(y[k], al2, nm2), t0, t1);
-      float e0 = fast_exp2(t0), e1 = fast_exp2(t1);
-      if (MASK) {
-        e0 = 2 * k <= kmax ? e0 : 0.0f;
-        e1 = 2 * k + 1 <= kmax ? e1 : 0.0f;
-      }
-      acc[k % 4] = add2(acc[k % 4], pk2(e0, e1));
-      w[e] = bf16x2(e0, e1);
-    }
-    *reinterpret_cast<uint4*>(prow + ((c ^ swz) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-  }
 }
 
 template <int T, int D>
@@ -462,15 +364,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           const CUtensorMap* vmap = plane == 8 ? &maps.v8 : &maps.v4;
           if (elect_one()) {
             mbar_arrive_expect_tx(&bars->v_full[vs], C::kVTile);
-            // V rows [token][d] as chunks of 64 values of d, each chunk 128 key rows (the
-            // load's block, or its two blocks at T = 64, a lone block copied twice)
-            const int jb[2] = {j0, (C::kBlocksPerLoad == 1 || j1 < 0) ? j0 : j1};
+            if constexpr (C::kBlocksPerLoad == 1) {
+              // one block of 128 keys as two V sub-tiles of 64 keys
+              const int vrow = static_cast<int>((grp * a.nb + j0) * D);
+              tma_load_2d(sV(vs), vmap, &bars->v_full[vs], 0, vrow);
+              tma_load_2d(sV(vs) + C::kVSub, vmap, &bars->v_full[vs], 64, vrow);
+            } else {
+              const int jb[2] = {j0, j1 >= 0 ? j1 : j0};
 #pragma unroll
-            for (int c = 0; c < D / 64; ++c)
-#pragma unroll
-              for (int h = 0; h < C::kBlocksPerLoad; ++h)
-                tma_load_2d(sV(vs) + c * C::kVChunk + h * T * 128, vmap, &bars->v_full[vs], 64 * c,
-                            static_cast<int>(grp * a.S + static_cast<int64_t>(jb[h]) * T));
+              for (int h = 0; h < 2; ++h)
+                tma_load_2d(sV(vs) + h * C::kVSub, vmap, &bars->v_full[vs], 0, static_cast<int>((grp * a.nb + jb[h]) * D));
+            }
           }
           __syncwarp();
           ++g;
@@ -544,18 +448,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = warp_wait(&bars->v_full[pr], (g / kPairs) & 1))) break;
           tc_fence_after();
           const uint64_t pdesc = sw128_desc(smem_u32(sP(pr)));
-          const uint64_t vdesc = sw128_mn_desc(smem_u32(sV(pr)), C::kVChunk);
+          const uint64_t vdesc = sw128_desc(smem_u32(sV(pr)));
           // the first P.V of a tile into an accumulator overwrites it: the tile's
           // loads l = 0 and l = 1 are the first of their pairs
           const bool first = l < kPairs;
           if (elect_one()) {
 #pragma unroll
             for (int s = 0; s < kKeys / 16; ++s) {
-              // P (K-major): +((s / 4) * sub-tile + (s % 4) * 32 bytes); V (N-major): + 16 key
-              // rows of 128 bytes; in the descriptors' 16-byte units
-              const uint64_t ad = pdesc + static_cast<uint64_t>((s % 4) * 32 >> 4) +
-                                  static_cast<uint64_t>(((s / 4) * C::kPSub) >> 4);
-              const uint64_t bd = vdesc + static_cast<uint64_t>((s * 16 * 128) >> 4);
+              // +((s / 4) * sub-tile + (s % 4) * 32 bytes) in the descriptor's 16-byte units
+              const uint64_t adv = static_cast<uint64_t>((s % 4) * 32 >> 4);
+              const uint64_t ad = pdesc + adv + static_cast<uint64_t>(((s / 4) * C::kPSub) >> 4);
+              const uint64_t bd = vdesc + adv + static_cast<uint64_t>(((s / 4) * C::kVSub) >> 4);
               mma_bf16_ss(tmem + o_col(pr), ad, bd, C::kIdescPV, (first && s == 0) ? 0u : 1u);
             }
             mma_commit(&bars->v_empty[pr]);

@@ -388,3 +388,9 @@ def tria_allocate(err, cost, budget: int) -> np.ndarray:
     out = np.zeros(H, np.int32)
     _check("tria_allocate", f(e.ctypes.data_as(P), c.ctypes.data_as(P), C, H, int(budget), out.ctypes.data_as(P)))
     return out
+
+
+def tria_prefill_gqa(enable: bool) -> bool:
+    """Allow (True) or forbid (False) the GQA-shared fused prefill; returns the previous setting."""
+    f = _typed("tria_prefill_gqa", [ctypes.c_int], ctypes.c_int)
+    return bool(f(1 if enable else 0))

@@ -50,6 +50,10 @@ WORKLOADS = {
                             T=128, seed=4, policy="maxctx"),
     "decode": Workload("decode", "decode", B=64, Hq=32, Hkv=8, D=128, S=32768, T=128,
                        seed=5, policy="decode"),
+    # the 8,192-token shapes with one (hi, keep) per KV head, shared by its 4 query heads
+    # (the case the GQA-shared prefill serves)
+    "llama_prefill_gqa": Workload("llama_prefill_gqa", "prefill", B=1, Hq=32, Hkv=8, D=128, S=8192,
+                                  T=64, seed=6, policy="llama_kv", k_outlier=4.0, k_outlier_frac=0.02),
 }
 
 
@@ -62,6 +66,12 @@ def policy(w: Workload) -> tuple[np.ndarray, np.ndarray]:
         return hi, keep
     hi = np.empty(w.Hq, np.int32)
     keep = np.empty(w.Hq, np.int32)
+    if w.policy == "llama_kv":         # hi ~ U{1..16}, keep ~ U{hi+1..64} per KV head
+        G = w.Hq // w.Hkv
+        for k in range(w.Hkv):
+            hi[k * G:(k + 1) * G] = rng.randint(1, 17)
+            keep[k * G:(k + 1) * G] = rng.randint(hi[k * G] + 1, 65)
+        return hi, keep
     for h in range(w.Hq):
         if w.policy == "llama":        # hi ~ U{1..16}, keep ~ U{hi+1..64}
             hi[h] = rng.randint(1, 17)

@@ -197,6 +197,15 @@ int tria_prefill(const void* Q, const tria_kv_cache* cache, const tria_dims* dim
                  const int32_t* hi, const int32_t* keep, void* O, float* LSE,
                  void* workspace, size_t workspace_bytes, void* stream);
 
+/* GQA-shared prefill (llmis.ru chapter 3.5, section 4: the query heads of a group
+ * read the same K and V). When Hq / Hkv is even and every pair of query heads
+ * (2k, 2k + 1) of the call has the same (hi, keep), the fused kernel serves both
+ * heads of a pair from one CTA, so each kept K/V block is brought on chip once for
+ * the two. Results are those of the per-head kernel. Enabled by default; this
+ * sets the process-wide choice (enable = 0: always per head) and returns the
+ * previous one. Host-only. */
+int tria_prefill_gqa(int enable);
+
 /* The two halves of tria_prefill, for callers that time or schedule them apart.
  * tria_prefill_prepare: Q codec (both planes) and the operand tiles built from
  * the cache (4-bit K expanded to one code per byte, V dequantised to bf16 and

@@ -112,10 +112,10 @@ def test_paged_decode_ragged_and_generation(T, oracle_mod):
         one.B = 1
         one.block_table = bt[b:b + 1].data_ptr()
         n = int(lens[b])
-        st = T.lib().tria_quantize_kv(K[b:b + 1, :, :n].contiguous().cuda().data_ptr(),
-                                      V[b:b + 1, :, :n].contiguous().cuda().data_ptr(), n, 0,
-                                      T.ctypes.byref(one), T._stream())
+        Kb, Vb = K[b:b + 1, :, :n].contiguous().cuda(), V[b:b + 1, :, :n].contiguous().cuda()   # alive until the copy ran
+        st = T.lib().tria_quantize_kv(Kb.data_ptr(), Vb.data_ptr(), n, 0, T.ctypes.byref(one), T._stream())
         assert st == 0
+        torch.cuda.synchronize()
     torch.cuda.synchronize()
     ws = torch.empty(T.tria_decode_workspace_bytes(B, Hq, Hkv, D, Tb, cap), dtype=torch.uint8, device="cuda")
     Kd, Vd = K.cuda(), V.cuda()
@@ -131,10 +131,10 @@ def test_paged_decode_ragged_and_generation(T, oracle_mod):
                 one.B = 1
                 one.block_table = bt[b:b + 1].data_ptr()
                 pos = int(lens[b])
-                st = T.lib().tria_quantize_kv(Kd[b:b + 1, :, pos:pos + 1].contiguous().data_ptr(),
-                                              Vd[b:b + 1, :, pos:pos + 1].contiguous().data_ptr(), 1, pos,
-                                              T.ctypes.byref(one), T._stream())
+                Kb, Vb = Kd[b:b + 1, :, pos:pos + 1].contiguous(), Vd[b:b + 1, :, pos:pos + 1].contiguous()
+                st = T.lib().tria_quantize_kv(Kb.data_ptr(), Vb.data_ptr(), 1, pos, T.ctypes.byref(one), T._stream())
                 assert st == 0
+                torch.cuda.synchronize()
             lens += 1
         q = seeded((B, Hq, D), 100 + step)
         Od, Ld = T.tria_decode(q.cuda(), cache, lens, hi, keep, workspace=ws)
