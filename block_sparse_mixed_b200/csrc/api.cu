@@ -474,6 +474,7 @@ int tria_prefill_attend(const tria_kv_cache* cache, const tria_dims* dims, const
   PrefillArgs a{};
   a.B = d.B; a.Hq = d.Hq; a.Hkv = d.Hkv; a.S = d.S; a.G = d.Hq / d.Hkv; a.nb = nb;
   a.ci = ci; a.k8_in_cache = d.D == 128;
+  a.cap = cache->capacity; a.cap8 = d.D == 128 ? cache->capacity : d.S;
   a.n_qtiles = (d.S + 127) / 128;
   a.n_units = d.B * d.Hq * a.n_qtiles;
   // Two query heads of a KV group share one CTA (and every K/V load) when their

@@ -80,8 +80,8 @@ struct PrepareArgs {
 
 struct PrefillArgs {
   int B, Hq, Hkv, S, G, nb;
-  CacheIndex ci;          // cache rows of the 8-bit K plane (D = 128) and of the K scales
-  bool k8_in_cache;       // the 8-bit K map covers the cache plane (D = 128) or the padded copy (D = 64)
+  int64_t cap;            // contiguous cache: rows per (b, kv head), scale arrays
+  int64_t cap8;           // rows per (b, kv head) behind the 8-bit K map (cap, or S when padded)
   int n_qtiles, n_units;
   float qk_log2;          // log2(e) / sqrt(D)
   const float* q8s;       // [B*Hq*S]
@@ -94,6 +94,8 @@ struct PrefillArgs {
   int* work;              // next query tile (dynamic scheduling); zero before the launch
   int hi[kMaxHeads];
   int keep[kMaxHeads];
+  CacheIndex ci;          // cache rows of the 8-bit K plane (D = 128) and of the K scales
+  bool k8_in_cache;       // the 8-bit K map covers the cache plane (D = 128) or the padded copy (D = 64)
 };
 
 struct PrefillMaps {

@@ -57,22 +57,18 @@ __device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
 // Softmax pass 1 over N keys of a row: y = float(acc) * s_k as packed pairs, and
 // the maximum over the visible keys (n <= kmax when MASK).
 // FP: S holds fp32 (the 4-bit plane's e4m3 product, an exact integer) instead of int32.
-// The int32 sums of the 8-bit plane are below 2^22 in magnitude (128 x 127 x 127), so
-// adding them to the bits of 1.5 * 2^23 gives the float 1.5 * 2^23 + acc exactly, and
-// one packed subtraction leaves acc: an integer add and half a float op per score in
-// place of a conversion on the transcendental unit, which the exponentials need.
+// (Converting the int32 sums through the bits of 1.5 * 2^23 and a packed subtraction,
+// instead of the int-to-float conversion, measured slower at T = 128.)
 template <int N, bool MASK, bool FP>
 __device__ __forceinline__ float scores_and_max(const uint32_t (&r)[N], uint64_t (&y)[N / 2], const float* sk,
                                                 int kmax) {
-  auto cv = [](uint32_t v) { return FP ? __uint_as_float(v) : __uint_as_float(v + 0x4B400000u); };
-  const uint64_t off2 = pk2(-12582912.0f, -12582912.0f);
-  auto cv2 = [&](uint64_t u) { return FP ? u : add2(u, off2); };
+  auto cv = [](uint32_t v) { return FP ? __uint_as_float(v) : __int2float_rn(static_cast<int>(v)); };
   float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
   for (int q = 0; q < N / 4; ++q) {
     const float4 s4 = *reinterpret_cast<const float4*>(sk + 4 * q);
-    const uint64_t u01 = cv2(pk2(cv(r[4 * q]), cv(r[4 * q + 1])));
-    const uint64_t u23 = cv2(pk2(cv(r[4 * q + 2]), cv(r[4 * q + 3])));
+    const uint64_t u01 = pk2(cv(r[4 * q]), cv(r[4 * q + 1]));
+    const uint64_t u23 = pk2(cv(r[4 * q + 2]), cv(r[4 * q + 3]));
     y[2 * q] = mul2(u01, pk2(s4.x, s4.y));
     y[2 * q + 1] = mul2(u23, pk2(s4.z, s4.w));
     float v0, v1, v2, v3;

@@ -112,7 +112,7 @@ struct Unit {
   int b, hq0, kvh, i0, nq;
 };
 
-// Units: (b, kv head, head pair, query tile), last query tiles first.
+// Units: (b, kv head, head pair, query tile), the last query tiles first.
 __device__ __forceinline__ Unit unit_of(const PrefillArgs& a, int w, int nqb) {
   Unit u;
   const int pairs = a.G / kHeads;
@@ -286,9 +286,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int jb[2] = {j0, (C::kBlocksPerLoad == 1 || j1 < 0) ? j0 : j1};
 #pragma unroll
             for (int h = 0; h < C::kBlocksPerLoad; ++h) {
-              int64_t crow = a.ci.block_row(u.b, u.kvh, jb[h]);
-              crow = crow < 0 ? 0 : crow;
-              const int64_t krow = k_in_cache ? crow : grp * a.S + static_cast<int64_t>(jb[h]) * T;
+              int64_t crow, krow;
+              if (a.ci.bt == nullptr) {     // contiguous cache
+                crow = grp * a.cap + static_cast<int64_t>(jb[h]) * T;
+                krow = grp * (plane == 8 ? a.cap8 : static_cast<int64_t>(a.S)) + static_cast<int64_t>(jb[h]) * T;
+              } else {                      // paged: the block's page (a bad page id reads page 0, reported)
+                crow = a.ci.block_row(u.b, u.kvh, jb[h]);
+                crow = crow < 0 ? 0 : crow;
+                krow = k_in_cache ? crow : grp * a.S + static_cast<int64_t>(jb[h]) * T;
+              }
               tma_load_2d(sK(ks) + h * T * kQKRowBytes, kmap, &bars->k_full[ks], 0, static_cast<int>(krow));
               bulk_load(sScale(ss) + h * T, ks_plane + crow, T * 4, &bars->sc_full[ss]);
             }

@@ -70,6 +70,8 @@ PREFILL = {
     "D128_T64": (2, 4, 2, 128, 64, 640, 12, [0, 2, 1, 3], [1, 5, 9, 4]),
     "D128_T128": (2, 4, 1, 128, 128, 768, 7, [1, 0, 2, 1], [3, 1, 4, 6]),
     "D64_T64": (1, 2, 1, 64, 64, 512, 9, [1, 2], [3, 5]),
+    # head pairs with equal boundaries: the GQA-shared kernel reads the paged cache
+    "D128_T64_gqa_pairs": (2, 4, 2, 128, 64, 640, 12, [2, 2, 0, 0], [5, 5, 9, 9]),
 }
 
 
