@@ -357,14 +357,17 @@ int tria_prefill_load_plan(int nb, int T, int hi, int keep, int32_t* plan, int64
       }
       ++n;
     };
+    const int64_t n0 = n;
     if (T == 128) {
       LoadPairs<1> lp;
       lp.init(i0, q, hi, keep);
       while (lp.next(j0, j1, plane)) emit();
+      if (n - n0 != load_count<1>(i0, q, hi, keep)) return TRIA_ERR_BOUNDS;   // the kernel's count
     } else {
       LoadPairs<2> lp;
       lp.init(i0, q, hi, keep);
       while (lp.next(j0, j1, plane)) emit();
+      if (n - n0 != load_count<2>(i0, q, hi, keep)) return TRIA_ERR_BOUNDS;
     }
   }
   *count = n;

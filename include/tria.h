@@ -173,7 +173,9 @@ int tria_count_tiles(int nb, int hi, int keep, int64_t* out);
  * -1 when j0 goes alone) and the plane, 8 or 4.
  * nb >= 0 blocks, T in {64, 128}, 0 <= hi <= keep. `plan` (host memory, may be
  * NULL) receives min(count, capacity) loads; *count receives the total.
- * Returns TRIA_ERR_INVALID_ARG on a bad argument or a NULL `count`. */
+ * Returns TRIA_ERR_INVALID_ARG on a bad argument or a NULL `count`, and
+ * TRIA_ERR_BOUNDS if a tile's walked load count differs from the closed-form count
+ * the kernel's producer uses (a self-check; it does not happen). */
 int tria_prefill_load_plan(int nb, int T, int hi, int keep, int32_t* plan, int64_t capacity, int64_t* count);
 
 /* Workspace bytes tria_prefill needs for `dims` (0 if dims are invalid). */
