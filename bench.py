@@ -254,6 +254,12 @@ def _ev():
     return torch.cuda.Event(enable_timing=True)
 
 
+# Device-side delay (clock cycles, about 2 ms) queued after each step's L2 flush and
+# before its first event: while the GPU waits, the host enqueues the whole step, so
+# the events measure the kernels back to back and not the host's launch overhead.
+HOST_LEAD_CYCLES = 4_000_000
+
+
 def _timed(step, steps, warmup, flush, clocks=None):
     """Run `step(times)` warmup + steps times (L2 flushed before each, outside the
     events); returns [steps, segments] ms from the events each step recorded."""
@@ -267,6 +273,7 @@ def _timed(step, steps, warmup, flush, clocks=None):
     try:
         for _ in range(steps):
             flush.zero_()
+            torch.cuda._sleep(HOST_LEAD_CYCLES)
             step(times)
         torch.cuda.synchronize()
     finally:
@@ -491,7 +498,7 @@ def run_gpu(args, rank, world, device):
 
     # Other workloads of the same path, timed in the same run (rows, not the headline).
     for name in args.legs:
-        if name == w.name:
+        if name == args.workload:
             continue
         lw = W.WORKLOADS[name]
         lclk = ClockSampler(torch.cuda.current_device())
@@ -688,6 +695,9 @@ def main():
         if args.heads > 0:
             ch["Hq"] = args.heads
             ch["Hkv"] = max(1, args.heads * w0.Hkv // w0.Hq)
+        # a slice is named apart from its workload, so that nothing recorded for the
+        # full workload (the DRAM traffic of profiles/traffic.md) is reported for it
+        ch["name"] = f"{w0.name}_slice"
         W.WORKLOADS[args.workload] = W.scaled(w0, **ch)
     w = W.WORKLOADS[args.workload]
 
