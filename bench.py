@@ -254,12 +254,6 @@ def _ev():
     return torch.cuda.Event(enable_timing=True)
 
 
-# Device-side delay (clock cycles, about 2 ms) queued after each step's L2 flush and
-# before its first event: while the GPU waits, the host enqueues the whole step, so
-# the events measure the kernels back to back and not the host's launch overhead.
-HOST_LEAD_CYCLES = 4_000_000
-
-
 def _timed(step, steps, warmup, flush, clocks=None):
     """Run `step(times)` warmup + steps times (L2 flushed before each, outside the
     events); returns [steps, segments] ms from the events each step recorded."""
@@ -273,7 +267,6 @@ def _timed(step, steps, warmup, flush, clocks=None):
     try:
         for _ in range(steps):
             flush.zero_()
-            torch.cuda._sleep(HOST_LEAD_CYCLES)
             step(times)
         torch.cuda.synchronize()
     finally:

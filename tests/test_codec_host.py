@@ -36,3 +36,68 @@ def test_division_free_scale_is_the_ieee_quotient_for_every_bf16():
             if rn32(q0 + e * r) != rn32(A / b):
                 bad.append(float(a))
         assert not bad, (b, bad[:5])
+
+
+# The codec's code quotients: q0 = RN(x r), e = RN(x - q0 s) (fused), q = RN(q0 + e r)
+# with r = RN(1 / s), then rint(q), against rint(RN(x / s)) clamped to the plane's
+# range (the oracle's IEEE division), for every pair of bf16 values 0 <= x <= amax
+# (negative x follow by symmetry: every step rounds to nearest). C with fmaf and
+# SSE single precision: IEEE binary32 operations, contraction off.
+_QUOTIENT_CHECK = r"""
+#include <math.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+static float f_of(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
+int main(void) {
+  const float lims[2] = {127.0f, 7.0f};
+  for (int pl = 0; pl < 2; ++pl) {
+    const float b = lims[pl];
+    long long bad_fast = 0, bad_tiny = 0, checked = 0;
+    float max_bad = 0.0f;
+#pragma omp parallel for schedule(dynamic, 64) reduction(+ : bad_fast, bad_tiny, checked) reduction(max : max_bad)
+    for (uint32_t ab = 1; ab < 0x7F80u; ++ab) {
+      const float A = f_of(ab << 16);
+      const float s = A / b;
+      const float r = 1.0f / s;
+      if (!(r < INFINITY)) continue;
+      for (uint32_t xb = 0; xb <= ab; ++xb) {
+        const float x = f_of(xb << 16);
+        const float q0 = x * r;
+        const float e = fmaf(-q0, s, x);
+        const float q = fmaf(e, r, q0);
+        float ref = rintf(x / s);
+        if (ref > b) ref = b;
+        ++checked;
+        if (rintf(q) != ref) {
+          if (A >= 0x1p-100f) ++bad_fast; else ++bad_tiny;
+          if (A > max_bad) max_bad = A;
+        }
+      }
+    }
+    printf("%d %lld %lld %lld %a\n", (int)b, checked, bad_fast, bad_tiny, max_bad);
+  }
+  return 0;
+}
+"""
+
+
+def test_division_free_codes_equal_the_ieee_quotient_codes(tmp_path):
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    assert gcc, "gcc is needed for this host check"
+    src = tmp_path / "quotients.c"
+    src.write_text(_QUOTIENT_CHECK)
+    exe = tmp_path / "quotients"
+    subprocess.run([gcc, "-O2", "-ffp-contract=off", "-fopenmp", str(src), "-o", str(exe), "-lm"], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    rows = [line.split() for line in out if line.strip()]
+    assert [int(r[0]) for r in rows] == [127, 7]
+    for lim, checked, bad_fast, bad_tiny, max_bad in rows:
+        # every (x, amax) pair with a finite reciprocal scale was visited
+        assert int(checked) > 5 * 10 ** 8
+        # the kernel takes the division-free path only for amax >= 2^-100, where
+        # it is exact; the few pairs it would get wrong lie far below (amax < 2^-117)
+        assert int(bad_fast) == 0, (lim, bad_fast)
+        assert float.fromhex(max_bad) < 2.0 ** -110, (lim, max_bad)

@@ -64,6 +64,20 @@ def test_codec_ties_and_scales_bit_exact(T, oracle_mod):
     ties32 = torch.stack(ties)
     ties = ties32.to(torch.bfloat16)
     assert torch.equal(ties.float(), ties32)   # bf16 holds every tie exactly
+    # Rows around the smallest maximum of the division-free path (2^-100) and far
+    # below it, down to bf16 subnormals, where the kernel divides exactly; the first
+    # two maxima (0x1.dep-118, 0x1.54p-120) with x = amax / 2 are pairs the
+    # division-free step would round wrongly.
+    gt = torch.Generator().manual_seed(321)
+    tiny = []
+    for amax in (2.0 ** -99, 2.0 ** -100, 2.0 ** -101, float.fromhex("0x1.dep-118"), float.fromhex("0x1.54p-120"),
+                 2.0 ** -126, 2.0 ** -130, 2.0 ** -133):
+        row = (torch.rand(D, generator=gt) * 2 - 1) * amax
+        row[0] = amax
+        row[1] = amax / 2
+        row[2] = -amax / 2
+        tiny.append(row)
+    ties = torch.cat([ties, torch.stack(tiny).to(torch.bfloat16)])
     g = torch.Generator().manual_seed(123)
     rnd = torch.randn((1 << 20, D), generator=g)
     rnd = rnd * torch.pow(2.0, torch.randint(-40, 41, (1 << 20, 1), generator=g).float())
