@@ -312,23 +312,25 @@ int tria_quantize_kv(const void* K, const void* V, int S, int start, const tria_
   if (S < 1 || start < 0 || static_cast<int64_t>(start) + S > cache->capacity) return TRIA_ERR_INVALID_ARG;
   if (!device_info().ok) return TRIA_ERR_UNSUPPORTED;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  for (int which = 0; which < 2; ++which) {
-    QuantArgs a{};
-    a.X = static_cast<const __nv_bfloat16*>(which == 0 ? K : V);
-    a.rows = static_cast<int64_t>(cache->B) * cache->Hkv * S;
-    a.cache = true;
-    a.ci = cache_index(*cache);
-    a.S = S;
-    a.start = start;
-    a.c8 = which == 0 ? cache->k8 : cache->v8;
-    a.ld8 = cache->D;
-    a.c4p = which == 0 ? cache->k4 : cache->v4;
-    a.s8 = which == 0 ? cache->k8_scale : cache->v8_scale;
-    a.s4 = which == 0 ? cache->k4_scale : cache->v4_scale;
-    const cudaError_t e = launch_quant_rows(a, cache->D, st);
-    if (e != cudaSuccess) return TRIA_ERR_CUDA;
-  }
-  return TRIA_OK;
+  // one launch for both tensors: K into the K planes, V (grid z = 1) into the V planes
+  QuantArgs a{};
+  a.X = static_cast<const __nv_bfloat16*>(K);
+  a.rows = static_cast<int64_t>(cache->B) * cache->Hkv * S;
+  a.cache = true;
+  a.ci = cache_index(*cache);
+  a.S = S;
+  a.start = start;
+  a.c8 = cache->k8;
+  a.ld8 = cache->D;
+  a.c4p = cache->k4;
+  a.s8 = cache->k8_scale;
+  a.s4 = cache->k4_scale;
+  a.X2 = static_cast<const __nv_bfloat16*>(V);
+  a.c8_2 = cache->v8;
+  a.c4p_2 = cache->v4;
+  a.s8_2 = cache->v8_scale;
+  a.s4_2 = cache->v4_scale;
+  return cuda_status(launch_quant_rows(a, cache->D, st));
 }
 
 int tria_count_tiles(int nb, int hi, int keep, int64_t* out) {

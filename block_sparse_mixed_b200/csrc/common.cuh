@@ -58,32 +58,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// try_wait with a suspend-time hint: the thread sleeps in hardware until the phase
-// completes or about `hint_ns` pass, instead of spinning on issue slots.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
-
 // Wait until the phase of `bar` with the given parity has completed. Returns
 // false (and raises *abort) when the block is aborting or the limit passes.
-// Waiting threads sleep (suspend hint), so they take no issue slots from the
-// warps that are computing; the abort flag and the clock are looked at only
-// when a sleep ends without the phase completing.
+// try_wait without a suspend-time hint: the hardware's own short wait inside each
+// try_wait, then the abort flag and the clock. (A 1 ms suspend hint, which takes the
+// waiting warp off the issue slots, measured 2-5% slower in the fused prefill and
+// 3% in the decode: the waiting warp resumes later after the phase completes.)
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int* err) {
-  constexpr uint32_t kSleepNs = 1000000;  // 1 ms
-  if (mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer();
   while (true) {
-    if (mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
     if (global_timer() - t0 > kWaitLimitNs) {
       *abort = 1;
@@ -99,11 +85,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // while the abort flag could be seen by one and not by the other.
 __device__ __forceinline__ bool mbar_wait_shared(uint64_t* bar, uint32_t parity, volatile int* abort,
                                                  int* err) {
-  constexpr uint32_t kSleepNs = 1000000;  // 1 ms
-  if (mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer();
   while (true) {
-    if (mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     if (global_timer() - t0 > kWaitLimitNs) {
       *abort = 1;
       atomicExch(err, TRIA_ERR_TIMEOUT);

@@ -48,7 +48,7 @@ struct CacheIndex {
 struct QuantArgs {
   const __nv_bfloat16* X;
   int64_t rows;
-  bool cache;
+  bool cache;         // rows of B * Hkv groups of S new tokens: grid (token blocks, groups, 1 or 2)
   CacheIndex ci;
   int64_t S;
   int64_t start;
@@ -59,6 +59,13 @@ struct QuantArgs {
   int ld4u;
   float* s8;
   float* s4;          // null: skip the 4-bit plane
+  int group0;         // cache path: group of grid row y = 0 (launches of at most 65,535 groups)
+  // cache path, grid z = 1: a second tensor (V) into its own planes, same layout
+  const __nv_bfloat16* X2;
+  int8_t* c8_2;
+  uint8_t* c4p_2;
+  float* s8_2;
+  float* s4_2;
 };
 
 struct PrepareArgs {

@@ -113,59 +113,5 @@ __device__ __forceinline__ void probs(const uint64_t (&y)[N / 2], uint64_t al2, 
   }
 }
 
-// In-place forms of the two passes, for a thread that holds all 128 keys of a load
-// (two halves of N = 64): pass 1 turns the raw S of a half into y = float(acc) * s_k
-// in the same registers and returns the maximum over the visible keys; pass 2 reads
-// y from them. Keeping one register per key keeps both halves within the budget.
-template <int N, bool MASK, bool FP>
-__device__ __forceinline__ float scores_and_max_inplace(uint32_t (&r)[N], const float* sk, int kmax) {
-  auto cv = [](uint32_t v) { return FP ? __uint_as_float(v) : __int2float_rn(static_cast<int>(v)); };
-  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-  for (int q = 0; q < N / 4; ++q) {
-    const float4 s4 = *reinterpret_cast<const float4*>(sk + 4 * q);
-    float v0, v1, v2, v3;
-    up2(mul2(pk2(cv(r[4 * q]), cv(r[4 * q + 1])), pk2(s4.x, s4.y)), v0, v1);
-    up2(mul2(pk2(cv(r[4 * q + 2]), cv(r[4 * q + 3])), pk2(s4.z, s4.w)), v2, v3);
-    r[4 * q] = __float_as_uint(v0);
-    r[4 * q + 1] = __float_as_uint(v1);
-    r[4 * q + 2] = __float_as_uint(v2);
-    r[4 * q + 3] = __float_as_uint(v3);
-    if (MASK) {
-      const int n = 4 * q;
-      v0 = n <= kmax ? v0 : -INFINITY;
-      v1 = n + 1 <= kmax ? v1 : -INFINITY;
-      v2 = n + 2 <= kmax ? v2 : -INFINITY;
-      v3 = n + 3 <= kmax ? v3 : -INFINITY;
-    }
-    mx[(q % 2) * 2] = max3(mx[(q % 2) * 2], v0, v1);
-    mx[(q % 2) * 2 + 1] = max3(mx[(q % 2) * 2 + 1], v2, v3);
-  }
-  return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-}
-
-template <int N, bool MASK>
-__device__ __forceinline__ void probs_inplace(const uint32_t (&r)[N], uint64_t al2, uint64_t nm2, int kmax,
-                                              uint8_t* prow, int swz, uint64_t (&acc)[4]) {
-#pragma unroll
-  for (int c = 0; c < N / 8; ++c) {
-    uint32_t w[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int k = 4 * c + e;
-      float t0, t1;
-      up2(fma2(pk2(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), al2, nm2), t0, t1);
-      float e0 = fast_exp2(t0), e1 = fast_exp2(t1);
-      if (MASK) {
-        e0 = 2 * k <= kmax ? e0 : 0.0f;
-        e1 = 2 * k + 1 <= kmax ? e1 : 0.0f;
-      }
-      acc[k % 4] = add2(acc[k % 4], pk2(e0, e1));
-      w[e] = bf16x2(e0, e1);
-    }
-    *reinterpret_cast<uint4*>(prow + ((c ^ swz) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-  }
-}
-
 }  // namespace pf
 }  // namespace tria
