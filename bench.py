@@ -152,8 +152,8 @@ class ClockSampler:
 def recorded_traffic(kernel: str, workload: str):
     """DRAM bytes per launch (read + write) of `kernel` on `workload`, from the ncu
     summary table in profiles/traffic.md, or None when there is no entry or the
-    kernel source has changed since the counters were taken (hash mismatch)."""
-    import hashlib
+    kernel's sources have changed since the counters were taken (hash mismatch: the
+    digest covers the kernel's file and the headers every kernel includes)."""
     import re
     table = ROOT / "profiles" / "traffic.md"
     if not table.exists():
@@ -163,11 +163,27 @@ def recorded_traffic(kernel: str, workload: str):
                      line)
         if not m or m.group(1) != kernel or m.group(2) != workload:
             continue
-        src = ROOT / "block_sparse_mixed_b200" / "csrc" / m.group(4)
-        if not src.exists() or hashlib.sha256(src.read_bytes()).hexdigest()[:12] != m.group(5):
+        if kernel_digest(m.group(4)) != m.group(5):
             return None
         return float(m.group(3))
     return None
+
+
+KERNEL_HEADERS = ("common.cuh", "kernels.h", "load_plan.cuh", "prefill_common.cuh")
+
+
+def kernel_digest(name: str):
+    """First 12 hex digits of the SHA-256 of a kernel source file followed by the shared
+    headers (in the order of KERNEL_HEADERS), or None if a file is missing."""
+    import hashlib
+    csrc = ROOT / "block_sparse_mixed_b200" / "csrc"
+    h = hashlib.sha256()
+    for f in (name,) + KERNEL_HEADERS:
+        p = csrc / f
+        if not p.exists():
+            return None
+        h.update(p.read_bytes())
+    return h.hexdigest()[:12]
 
 
 # ---------------------------------------------------------------- accounting
