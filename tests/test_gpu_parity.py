@@ -113,6 +113,33 @@ def test_cache_write_and_append_bit_exact(T, oracle_mod):
         assert (cache.plane(p + "8")[:, :, 201:].cpu().view(torch.uint8) == 0x5A).all()  # untouched
 
 
+def test_cache_write_more_groups_than_one_launch_bit_exact(T, oracle_mod):
+    """A one-token write into B * Hkv = 65,544 (batch, KV head) groups: more than the
+    65,535 grid rows of one codec launch, so the write is split over two launches."""
+    B, Hkv, D, Tb, cap, start = 8193, 8, 64, 64, 64, 37
+    cache = T.CompressedKVCache(B, Hkv, D, Tb, cap)
+    cache.buffer.fill_(0x5A)
+    K, V = seeded((B, Hkv, 1, D), 11), seeded((B, Hkv, 1, D), 12)
+    T.tria_quantize_kv(K.cuda(), V.cuda(), cache, start=start)
+    torch.cuda.synchronize()
+    for X, p in ((K, "k"), (V, "v")):
+        r8, rs8, r4, rs4 = oracle_mod.quantize_rows(X, D)
+        got8 = cache.plane(p + "8")[:, :, start].cpu().numpy().reshape(-1, D)
+        got4 = cache.plane(p + "4")[:, :, start].cpu().numpy().reshape(-1, D // 2)
+        assert np.array_equal(got8, r8)
+        assert np.array_equal(got4, oracle_mod.pack_int4(r4))
+        assert np.array_equal(cache.plane(p + "8_scale")[:, :, start].cpu().numpy().reshape(-1).view(np.uint32),
+                              rs8.view(np.uint32))
+        assert np.array_equal(cache.plane(p + "4_scale")[:, :, start].cpu().numpy().reshape(-1).view(np.uint32),
+                              rs4.view(np.uint32))
+        # the rows next to the written token are untouched, in the first and the last group
+        for b in (0, B - 1):
+            assert (cache.plane(p + "8")[b, :, start - 1].cpu().view(torch.uint8) == 0x5A).all()
+            assert (cache.plane(p + "8")[b, :, start + 1].cpu().view(torch.uint8) == 0x5A).all()
+    del cache
+    torch.cuda.empty_cache()
+
+
 # ---------------------------------------------------------------- prefill
 
 def run_prefill(T, Q, K, V, Tb, hi, keep, cap=None):
