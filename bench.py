@@ -72,8 +72,9 @@ class ClockSampler:
     NVML is not importable."""
 
     # NVML clock-event reason bits
-    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
-               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+    REASONS = {0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -95,6 +96,9 @@ class ClockSampler:
             self.mx.append(float(mx))
             bits = int(get_reasons(h))
             self.reasons.update(name for bit, name in self.REASONS.items() if bits & bit)
+            other = bits & ~(0x1 | sum(self.REASONS))   # 0x1: idle
+            if other:
+                self.reasons.add(f"other_{other:#x}")
             self._stop.wait(0.005)
 
     def _run_smi(self):
@@ -351,21 +355,29 @@ def prefill_leg(tria, w, args, flush, stream, clocks=None, e2e=True):
            "codec_bytes": 2 * (K.numel() * 2) + 2 * (K.numel() + K.numel() // 2) + 4 * 4 * K.numel() // w.D,
            "launches_per_step": 2 + 2 + 1 + 2}
     if e2e:
+        # The user's call from host memory: tria_prefill_host writes the cache and runs the
+        # prefill group by group, its copies in and out overlapping the kernels; then the
+        # last token's decode from its host query row.
         hQ, hK, hV = (t.cpu().pin_memory() for t in (Q, K, V))
+        hq_last = q_last.cpu().pin_memory()
         hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
         hL = torch.empty(LSE.shape, dtype=LSE.dtype).pin_memory()
         hOd = torch.empty(Od.shape, dtype=Od.dtype).pin_memory()
+        del O, LSE, ws
+        torch.cuda.empty_cache()
+        host_prefill = tria.HostPrefill(w.B, w.Hq, w.Hkv, w.S, w.D, w.T, device=device)
 
         def e2e_step():
-            Q.copy_(hQ, non_blocking=True); K.copy_(hK, non_blocking=True); V.copy_(hV, non_blocking=True)
-            tria.tria_quantize_kv(K, V, cache)
-            tria.tria_prefill(Q, cache, hi, keep, workspace=ws, O=O, LSE=LSE)
-            q_last.copy_(Q[:, :, w.S - 1])
+            host_prefill(hQ, hK, hV, cache, hi, keep, hO, hL, stream=stream)
+            q_last.copy_(hq_last, non_blocking=True)
             tria.tria_decode(q_last, cache, kv_len, hi, keep, workspace=dws, O=Od, LSE=Ld)
-            hO.copy_(O, non_blocking=True); hL.copy_(LSE, non_blocking=True); hOd.copy_(Od, non_blocking=True)
+            hOd.copy_(Od, non_blocking=True)
 
         out["e2e_ms"] = _e2e(e2e_step, args.steps, args.warmup, flush, stream)
-        out["h2d"] = sum(t.numel() * t.element_size() for t in (hQ, hK, hV))
+        st = tria.tria_workspace_status(host_prefill.workspace)
+        if st != 0:
+            raise RuntimeError(f"{w.name}: device-side error in the host-buffer prefill: {tria.tria_status_string(st)}")
+        out["h2d"] = sum(t.numel() * t.element_size() for t in (hQ, hK, hV, hq_last))
         out["d2h"] = sum(t.numel() * t.element_size() for t in (hO, hL, hOd))
     return out
 

@@ -18,7 +18,8 @@ ROOT = PKG.parent
 CSRC = PKG / "csrc"
 OUT = PKG / "libtria.so"
 BUILD = ROOT / "_build"
-SOURCES = ["api.cu", "quant.cu", "prefill_sm100.cu", "decode.cu", "decode_static.cu", "calib.cu", "prefill_gqa_sm100.cu"]
+SOURCES = ["api.cu", "quant.cu", "prefill_sm100.cu", "decode.cu", "decode_static.cu", "calib.cu", "prefill_gqa_sm100.cu",
+           "pipeline.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC", "-I", str(ROOT / "include"), "-I", str(CSRC)]

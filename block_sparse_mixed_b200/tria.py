@@ -394,3 +394,46 @@ def tria_prefill_gqa(enable: bool) -> bool:
     """Allow (True) or forbid (False) the GQA-shared fused prefill; returns the previous setting."""
     f = _typed("tria_prefill_gqa", [ctypes.c_int], ctypes.c_int)
     return bool(f(1 if enable else 0))
+
+
+def _host_ptr(t: torch.Tensor) -> ctypes.c_void_p:
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError("expected a contiguous host tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def tria_prefill_host_staging_bytes(B, Hq, Hkv, S, D, T) -> int:
+    f = _typed("tria_prefill_host_staging_bytes", [ctypes.POINTER(tria_dims)], ctypes.c_size_t)
+    return int(f(ctypes.byref(tria_dims(B, Hq, Hkv, S, D, T))))
+
+
+def tria_prefill_host_workspace_bytes(B, Hq, Hkv, S, D, T) -> int:
+    f = _typed("tria_prefill_host_workspace_bytes", [ctypes.POINTER(tria_dims)], ctypes.c_size_t)
+    return int(f(ctypes.byref(tria_dims(B, Hq, Hkv, S, D, T))))
+
+
+class HostPrefill:
+    """Device buffers and the two copy streams of tria_prefill_host for one shape, kept
+    across calls (the library itself allocates nothing)."""
+
+    def __init__(self, B, Hq, Hkv, S, D, T, device="cuda"):
+        self.dims = tria_dims(B, Hq, Hkv, S, D, T)
+        self.shape = (B, Hq, Hkv, S, D, T)
+        self.staging = _aligned_empty(tria_prefill_host_staging_bytes(*self.shape), device)
+        self.workspace = _aligned_empty(tria_prefill_host_workspace_bytes(*self.shape), device)
+        self.copy_in = torch.cuda.Stream(device=device)
+        self.copy_out = torch.cuda.Stream(device=device)
+
+    def __call__(self, hQ, hK, hV, cache: CompressedKVCache, hi, keep, hO, hLSE, stream=None):
+        """Cache write and prefill from host tensors hQ/hK/hV into host hO/hLSE (queued on
+        `stream`; synchronise it before reading hO)."""
+        P = ctypes.c_void_p
+        f = _typed("tria_prefill_host", [P, P, P, ctypes.POINTER(tria_kv_cache), ctypes.POINTER(tria_dims), P, P, P,
+                                         P, P, ctypes.c_size_t, P, ctypes.c_size_t, P, P, P], ctypes.c_int)
+        hi_a, keep_a = _host_i32(hi), _host_i32(keep)
+        _check("tria_prefill_host", f(
+            _host_ptr(hQ), _host_ptr(hK), _host_ptr(hV), ctypes.byref(cache.struct), ctypes.byref(self.dims),
+            hi_a.ctypes.data_as(P), keep_a.ctypes.data_as(P), _host_ptr(hO), _host_ptr(hLSE),
+            _dev_ptr(self.staging), self.staging.numel(), _dev_ptr(self.workspace), self.workspace.numel(),
+            _stream(stream), _stream(self.copy_in), _stream(self.copy_out)))
+        return hO, hLSE

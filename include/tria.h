@@ -208,6 +208,38 @@ int tria_prefill(const void* Q, const tria_kv_cache* cache, const tria_dims* dim
  * previous one. Host-only. */
 int tria_prefill_gqa(int enable);
 
+/* Prefill of a prompt held in host memory: the cache write of tokens [0, S) of K and
+ * V (as tria_quantize_kv) and the fused prefill of Q (as tria_prefill, the same
+ * computation: rit.work TriAttention page, section "Как калибровка распределяет
+ * вычисления между головами", last paragraph), with the copies in and out overlapped
+ * with the kernels. The work is split by (batch, KV head) group: group g's K, V and
+ * its Hq/Hkv query heads' Q are copied in on copy_in_stream while group g - 1's
+ * kernels run on `stream` and group g - 2's O and LSE are copied out on
+ * copy_out_stream, through two slots of `staging`.
+ *   hQ, hK, hV    host bf16, [B,Hq,S,D] and [B,Hkv,S,D]; page-locked memory lets the
+ *                 copies overlap (pageable memory works, serialised by the runtime).
+ *   hO, hLSE      host bf16 [B,Hq,S,D] and fp32 [B,Hq,S], written by the call.
+ *   cache         contiguous cache (no block table) with B, Hkv, D, T of dims and
+ *                 capacity >= S; its rows [0, S) of every group are written.
+ *   hi, keep      host int32 [Hq], as tria_prefill.
+ *   staging       device, 256-byte aligned, >= tria_prefill_host_staging_bytes(dims).
+ *   workspace     device, 256-byte aligned, >= tria_prefill_host_workspace_bytes(dims)
+ *                 (the prefill workspace of one group); its status word is read with
+ *                 tria_workspace_status.
+ *   streams       three distinct streams. The call returns once everything is queued;
+ *                 `stream` completes after the last copy out, so synchronising it (or
+ *                 an event recorded on it after the call) makes hO and hLSE readable.
+ * Returns TRIA_ERR_UNSUPPORTED for a paged cache, TRIA_ERR_INVALID_ARG for a
+ * missing pointer, equal streams, a small buffer or dims that disagree with the
+ * cache; the per-group calls' own checks and status codes otherwise. */
+size_t tria_prefill_host_staging_bytes(const tria_dims* dims);
+size_t tria_prefill_host_workspace_bytes(const tria_dims* dims);
+int tria_prefill_host(const void* hQ, const void* hK, const void* hV, const tria_kv_cache* cache,
+                      const tria_dims* dims, const int32_t* hi, const int32_t* keep,
+                      void* hO, float* hLSE, void* staging, size_t staging_bytes,
+                      void* workspace, size_t workspace_bytes, void* stream,
+                      void* copy_in_stream, void* copy_out_stream);
+
 /* The two halves of tria_prefill, for callers that time or schedule them apart.
  * tria_prefill_prepare: Q codec (both planes) and the operand tiles built from
  * the cache (4-bit K expanded to one code per byte, V dequantised to bf16 and

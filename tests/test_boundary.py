@@ -23,7 +23,7 @@ EXPECTED = {
     "tria_decode_static", "tria_decode_static_status", "tria_workspace_status",
     "tria_paged_cache_bytes", "tria_paged_cache_init", "tria_cache_status",
     "tria_calibration_costs", "tria_calibrate_workspace_bytes", "tria_calibrate", "tria_allocate",
-    "tria_prefill_gqa",
+    "tria_prefill_gqa", "tria_prefill_host_staging_bytes", "tria_prefill_host_workspace_bytes", "tria_prefill_host",
 }
 
 
