@@ -258,6 +258,10 @@ DECODE_CASES = {
     "g16": (1, 16, 1, 128, 64, 1024, [777], [(h % 4, 2 + h) for h in range(16)]),
     "g12_t128": (1, 12, 1, 128, 128, 2048, [1999], [(h % 5, 1 + 2 * h) for h in range(12)]),
     "t128_d64_g8": (2, 16, 2, 64, 128, 1536, [1536, 700], [((3 * h) % 4, 2 + (h % 7)) for h in range(16)]),
+    # one long sequence and one KV group: about 65 kept blocks, one work item each, so
+    # the group has more than 256 partials and the merge splits its columns over CTAs
+    "long_one_group_t128": (1, 4, 1, 128, 128, 8192, [8192], [(2, 60), (5, 64), (0, 40), (9, 63)]),
+    "long_one_group_d64": (1, 2, 1, 64, 64, 4096, [4000], [(1, 62), (3, 50)]),
 }
 
 
