@@ -201,7 +201,12 @@ def prefill_work(w: W.Workload, hi, keep, tria):
         n4 += c[1]
     tiles = w.B * (n8 + n4)
     per = 2 * w.T * w.T * w.D
+    # diagonal tiles (one per query block, always 8-bit) count whole, as executed; the
+    # causal count keeps only their T (T + 1) / 2 visible (query, key) pairs
+    diag = w.B * len(hi) * w.nb
+    causal = (tiles - diag) * per + diag * per * (w.T + 1) / (2 * w.T)
     return {"tiles_int8": w.B * n8, "tiles_int4": w.B * n4, "ops_int8": tiles * per, "flop_bf16": tiles * per,
+            "tiles_diagonal": diag, "ops_int8_causal": causal, "flop_bf16_causal": causal,
             "kept_fraction": (n8 + n4) / (len(hi) * w.nb * (w.nb + 1) / 2), "int4_share": n4 / max(1, n8 + n4)}
 
 
@@ -447,7 +452,9 @@ def prefill_rows(w, r, peaks):
                         "frac_hbm": r["codec_bytes"] / (r["quantize_kv_ms"] / 1e3) / 1e9 / hbm},
         "prefill": {"ms": p_ms, "prepare_ms": r["prepare_ms"], "attend_ms": r["attend_ms"],
                     "attend_ms_min": r["attend_ms_min"], "TOPS_kept": achieved, "frac_roofline": achieved / peak,
-                    "TOPS_kept_whole_call": ops / (p_ms / 1e3) / 1e12, **r["work"]},
+                    "TOPS_kept_whole_call": ops / (p_ms / 1e3) / 1e12,
+                    "TOPS_kept_causal": (r["work"]["ops_int8_causal"] + r["work"]["flop_bf16_causal"])
+                    / (r["attend_ms"] / 1e3) / 1e12, **r["work"]},
         "decode_last_token": {"ms": r["decode_ms"], "kept_bytes": r["decode_bytes"],
                               "GB/s": r["decode_bytes"] / (r["decode_ms"] / 1e3) / 1e9},
     }
