@@ -101,3 +101,54 @@ def test_division_free_codes_equal_the_ieee_quotient_codes(tmp_path):
         # it is exact; the few pairs it would get wrong lie far below (amax < 2^-117)
         assert int(bad_fast) == 0, (lim, bad_fast)
         assert float.fromhex(max_bad) < 2.0 ** -110, (lim, max_bad)
+
+
+# The codec's reciprocal of a scale: a first guess r0 (the hardware approximation,
+# documented within 1 ulp of 1/s), then e = RN(1 - s r0) and r = RN(r0 + e r0), both
+# fused. For every scale s = RN(amax / b) of a bf16 row maximum amax >= 2^-100 (the
+# division-free path) and every r0 within 3 ulps of RN(1/s), r must be RN(1/s).
+_RECIPROCAL_CHECK = r"""
+#include <math.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+static float f_of(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
+static uint32_t u_of(float f) { uint32_t u; memcpy(&u, &f, 4); return u; }
+int main(void) {
+  const float lims[2] = {127.0f, 7.0f};
+  for (int pl = 0; pl < 2; ++pl) {
+    long long bad = 0, checked = 0;
+    for (uint32_t ab = 1; ab < 0x7F80u; ++ab) {
+      const float A = f_of(ab << 16);
+      if (!(A >= 0x1p-100f)) continue;
+      const float s = A / lims[pl];
+      const float R = 1.0f / s;
+      for (int k = -3; k <= 3; ++k) {
+        const float r0 = f_of(u_of(R) + k);
+        const float e = fmaf(-s, r0, 1.0f);
+        ++checked;
+        if (fmaf(e, r0, r0) != R) ++bad;
+      }
+    }
+    printf("%d %lld %lld\n", (int)lims[pl], checked, bad);
+  }
+  return 0;
+}
+"""
+
+
+def test_newton_step_gives_the_correctly_rounded_reciprocal_of_every_scale(tmp_path):
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    assert gcc, "gcc is needed for this host check"
+    src = tmp_path / "reciprocal.c"
+    src.write_text(_RECIPROCAL_CHECK)
+    exe = tmp_path / "reciprocal"
+    subprocess.run([gcc, "-O2", "-ffp-contract=off", str(src), "-o", str(exe), "-lm"], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    rows = [line.split() for line in out if line.strip()]
+    assert [int(r[0]) for r in rows] == [127, 7]
+    for lim, checked, bad in rows:
+        assert int(checked) == 7 * 29184, (lim, checked)   # 29,184 maxima of bf16 in [2^-100, max]
+        assert int(bad) == 0, (lim, bad)
