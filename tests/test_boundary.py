@@ -152,6 +152,48 @@ def test_host_validation_rejects_bad_arguments(L):
                                 None) == tria.TRIA_ERR_INVALID_ARG
 
 
+def test_host_prefill_validation_before_any_cuda_call(L):
+    """tria_prefill_host checks every argument on the host before it creates an event
+    or queues a copy, so these calls return at once, here without a GPU."""
+    P = ctypes.c_void_p
+    f = L.tria_prefill_host
+    f.argtypes = [P, P, P, ctypes.POINTER(tria.tria_kv_cache), ctypes.POINTER(tria.tria_dims), P, P, P, P,
+                  P, ctypes.c_size_t, P, ctypes.c_size_t, P, P, P]
+    f.restype = ctypes.c_int
+    for fn in ("tria_prefill_host_staging_bytes", "tria_prefill_host_workspace_bytes"):
+        getattr(L, fn).argtypes = [ctypes.POINTER(tria.tria_dims)]
+        getattr(L, fn).restype = ctypes.c_size_t
+    c = _fake_cache(B=1, Hkv=2, D=128, T=64, cap=512)
+    d = tria.tria_dims(1, 4, 2, 512, 128, 64)
+    i32 = lambda v: np.ascontiguousarray(v, np.int32)
+    hi, keep = i32([1, 2, 1, 2]), i32([3, 5, 3, 5])
+    host = P(1 << 30)
+    staging, ws = P(1 << 41), P(1 << 42)
+    sbytes = L.tria_prefill_host_staging_bytes(ctypes.byref(d))
+    wbytes = L.tria_prefill_host_workspace_bytes(ctypes.byref(d))
+    # two slots of (Q of 2 heads, K, V, O of 2 heads, LSE of 2 heads) at S = 512, D = 128
+    assert sbytes == 2 * (2 * 262144 + 2 * 131072 + 4096)
+    assert wbytes == tria.tria_prefill_workspace_bytes(1, 2, 1, 512, 128, 64) > 0
+    s1, s2, s3 = P(1), P(2), P(3)
+
+    def call(hQ=host, cache=c, dims=d, st=staging, sb=sbytes, wb=wbytes, streams=(s1, s2, s3)):
+        return f(hQ, host, host, ctypes.byref(cache), ctypes.byref(dims), hi.ctypes.data_as(P),
+                 keep.ctypes.data_as(P), host, host, st, sb, ws, wb, *streams)
+
+    assert call(hQ=None) == tria.TRIA_ERR_INVALID_ARG
+    assert call(streams=(s1, s2, s2)) == tria.TRIA_ERR_INVALID_ARG          # one stream for both copies
+    assert call(streams=(s1, s1, s3)) == tria.TRIA_ERR_INVALID_ARG          # copies on the compute stream
+    assert call(st=P((1 << 41) + 16)) == tria.TRIA_ERR_INVALID_ARG          # staging not 256-byte aligned
+    assert call(sb=sbytes - 1) == tria.TRIA_ERR_INVALID_ARG
+    assert call(wb=wbytes - 1) == tria.TRIA_ERR_INVALID_ARG
+    assert call(dims=tria.tria_dims(1, 4, 2, 1024, 128, 64)) == tria.TRIA_ERR_INVALID_ARG   # S > capacity
+    assert call(dims=tria.tria_dims(1, 4, 1, 512, 128, 64)) == tria.TRIA_ERR_INVALID_ARG    # Hkv differs
+    paged = tria.tria_kv_cache()
+    ctypes.memmove(ctypes.byref(paged), ctypes.byref(c), ctypes.sizeof(c))
+    paged.block_table = P(1 << 43)
+    assert call(cache=paged) == tria.TRIA_ERR_UNSUPPORTED
+
+
 def test_calibration_costs_match_oracle(L):
     from oracle import calibration as cal
     for nb, T, D in ((8, 64, 128), (37, 128, 64), (1, 64, 64)):
