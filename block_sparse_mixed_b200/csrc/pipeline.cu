@@ -7,15 +7,18 @@
 // query heads' Q rows in, their O and LSE rows out. Every group is independent (its
 // cache rows, its query heads and its outputs are its own), so group g's kernels run
 // while group g + 1's inputs are copied in and group g - 1's outputs are copied out,
-// through two staging slots in device memory.
+// through two to four staging slots in device memory (as many as the caller's
+// staging buffer holds).
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <algorithm>
 
 #include "tria.h"
 
 namespace {
 
-constexpr int kSlots = 2;
+constexpr int kMinSlots = 2, kMaxSlots = 4;
 
 struct Slots {
   size_t q, kv, o, lse, slot;   // bytes of each buffer of one slot, and of one whole slot
@@ -68,7 +71,7 @@ extern "C" {
 
 size_t tria_prefill_host_staging_bytes(const tria_dims* dims) {
   if (!dims_ok(dims)) return 0;
-  return kSlots * slot_sizes(*dims).slot;
+  return kMinSlots * slot_sizes(*dims).slot;
 }
 
 size_t tria_prefill_host_workspace_bytes(const tria_dims* dims) {
@@ -92,7 +95,9 @@ int tria_prefill_host(const void* hQ, const void* hK, const void* hV, const tria
   if (cache->B != d.B || cache->Hkv != d.Hkv || cache->D != d.D || cache->T != d.T || cache->capacity < d.S)
     return TRIA_ERR_INVALID_ARG;
   const Slots sz = slot_sizes(d);
-  if (staging_bytes < kSlots * sz.slot) return TRIA_ERR_INVALID_ARG;
+  if (staging_bytes < kMinSlots * sz.slot) return TRIA_ERR_INVALID_ARG;
+  // a larger staging buffer buys more slots: the copies in run further ahead
+  const int slots = static_cast<int>(std::min<size_t>(kMaxSlots, staging_bytes / sz.slot));
   const tria_dims gd = group_dims(d);
   const size_t ws_need = tria_prefill_workspace_bytes(&gd);
   if (ws_need == 0) return TRIA_ERR_UNSUPPORTED;
@@ -114,7 +119,7 @@ int tria_prefill_host(const void* hQ, const void* hK, const void* hV, const tria
 
   // Events: the start of the call on `stream`; per slot, inputs copied in, inputs
   // consumed (after the preparation), outputs written, outputs copied out.
-  cudaEvent_t ev[1 + 4 * kSlots] = {};
+  cudaEvent_t ev[1 + 4 * kMaxSlots] = {};
   int status = TRIA_OK;
   for (auto& e : ev)
     if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) status = TRIA_ERR_CUDA;
@@ -138,11 +143,11 @@ int tria_prefill_host(const void* hQ, const void* hK, const void* hV, const tria
     ok(cudaStreamWaitEvent(so, start, 0));
 
   for (int gi = 0; gi < groups && status == TRIA_OK; ++gi) {
-    const int s = gi % kSlots;
+    const int s = gi % slots;
     const int b = gi / d.Hkv, kvh = gi % d.Hkv;
     const size_t qrow0 = static_cast<size_t>(b) * d.Hq + static_cast<size_t>(kvh) * G;   // first query head row
-    // inputs of group gi into slot s, once group gi - 2 has consumed it
-    if (gi >= kSlots && !ok(cudaStreamWaitEvent(si, in_free(s), 0))) break;
+    // inputs of group gi into slot s, once group gi - slots has consumed it
+    if (gi >= slots && !ok(cudaStreamWaitEvent(si, in_free(s), 0))) break;
     if (!ok(cudaMemcpyAsync(k_of(s), static_cast<const uint8_t*>(hK) + gi * kvbytes, kvbytes, cudaMemcpyHostToDevice, si)))
       break;
     if (!ok(cudaMemcpyAsync(v_of(s), static_cast<const uint8_t*>(hV) + gi * kvbytes, kvbytes, cudaMemcpyHostToDevice, si)))
@@ -152,9 +157,9 @@ int tria_prefill_host(const void* hQ, const void* hK, const void* hV, const tria
       break;
     if (!ok(cudaEventRecord(in_ready(s), si))) break;
     // kernels of group gi: cache write, preparation, fused prefill into slot s's outputs
-    // (once group gi - 2's outputs have been copied out of it)
+    // (once group gi - slots' outputs have been copied out of it)
     if (!ok(cudaStreamWaitEvent(sc, in_ready(s), 0))) break;
-    if (gi >= kSlots && !ok(cudaStreamWaitEvent(sc, out_free(s), 0))) break;
+    if (gi >= slots && !ok(cudaStreamWaitEvent(sc, out_free(s), 0))) break;
     const tria_kv_cache gc = group_cache(*cache, gi);
     if (!ok_t(tria_quantize_kv(k_of(s), v_of(s), d.S, 0, &gc, sc))) break;
     if (!ok_t(tria_prefill_prepare(q_of(s), &gc, &gd, workspace, workspace_bytes, sc))) break;

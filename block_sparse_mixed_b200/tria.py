@@ -416,10 +416,12 @@ class HostPrefill:
     """Device buffers and the two copy streams of tria_prefill_host for one shape, kept
     across calls (the library itself allocates nothing)."""
 
-    def __init__(self, B, Hq, Hkv, S, D, T, device="cuda"):
+    def __init__(self, B, Hq, Hkv, S, D, T, device="cuda", slots=2):
+        """slots: staging slots (2 to 4); with more, the copies in run further ahead."""
         self.dims = tria_dims(B, Hq, Hkv, S, D, T)
         self.shape = (B, Hq, Hkv, S, D, T)
-        self.staging = _aligned_empty(tria_prefill_host_staging_bytes(*self.shape), device)
+        per_slot = tria_prefill_host_staging_bytes(*self.shape) // 2
+        self.staging = _aligned_empty(per_slot * max(2, min(4, int(slots))), device)
         self.workspace = _aligned_empty(tria_prefill_host_workspace_bytes(*self.shape), device)
         self.copy_in = torch.cuda.Stream(device=device)
         self.copy_out = torch.cuda.Stream(device=device)

@@ -215,14 +215,16 @@ int tria_prefill_gqa(int enable);
  * with the kernels. The work is split by (batch, KV head) group: group g's K, V and
  * its Hq/Hkv query heads' Q are copied in on copy_in_stream while group g - 1's
  * kernels run on `stream` and group g - 2's O and LSE are copied out on
- * copy_out_stream, through two slots of `staging`.
+ * copy_out_stream, through the slots of `staging`.
  *   hQ, hK, hV    host bf16, [B,Hq,S,D] and [B,Hkv,S,D]; page-locked memory lets the
  *                 copies overlap (pageable memory works, serialised by the runtime).
  *   hO, hLSE      host bf16 [B,Hq,S,D] and fp32 [B,Hq,S], written by the call.
  *   cache         contiguous cache (no block table) with B, Hkv, D, T of dims and
  *                 capacity >= S; its rows [0, S) of every group are written.
  *   hi, keep      host int32 [Hq], as tria_prefill.
- *   staging       device, 256-byte aligned, >= tria_prefill_host_staging_bytes(dims).
+ *   staging       device, 256-byte aligned, >= tria_prefill_host_staging_bytes(dims)
+ *                 (two slots); a buffer of k slots' bytes, k <= 4, lets the copies in
+ *                 run k - 1 groups ahead of the kernels.
  *   workspace     device, 256-byte aligned, >= tria_prefill_host_workspace_bytes(dims)
  *                 (the prefill workspace of one group); its status word is read with
  *                 tria_workspace_status.
