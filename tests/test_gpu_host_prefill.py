@@ -7,7 +7,8 @@ it writes and the O and LSE it copies out must equal that path's bit for bit (wi
 the same fused kernel: per-head policies that differ within every head pair, or
 pairs that agree in every group so both paths take the GQA-shared kernel), and O
 and LSE must match the oracle on sampled rows. Shapes cover several groups per
-sequence, B > 1, both block sizes, and more groups than staging slots.
+sequence, B > 1, both block sizes, two to four staging slots and more groups than
+slots.
 """
 import numpy as np
 import pytest
@@ -33,16 +34,16 @@ def seeded(shape, seed):
 
 
 CASES = {
-    # B, Hq, Hkv, S, D, T, per-query-head (hi, keep)
-    "per_head_t64": (2, 8, 2, 1024, 128, 64, [(1, 3), (2, 9), (0, 4), (3, 5), (1, 2), (4, 12), (2, 2), (0, 7)]),
-    "pairs_t128": (1, 8, 4, 1280, 128, 128, [(1, 4), (1, 4), (2, 6), (2, 6), (0, 3), (0, 3), (3, 8), (3, 8)]),
-    "d64_g1_t64": (3, 2, 2, 576, 64, 64, [(1, 5), (2, 3)]),
+    # B, Hq, Hkv, S, D, T, per-query-head (hi, keep), staging slots
+    "per_head_t64": (2, 8, 2, 1024, 128, 64, [(1, 3), (2, 9), (0, 4), (3, 5), (1, 2), (4, 12), (2, 2), (0, 7)], 2),
+    "pairs_t128": (1, 8, 4, 1280, 128, 128, [(1, 4), (1, 4), (2, 6), (2, 6), (0, 3), (0, 3), (3, 8), (3, 8)], 3),
+    "d64_g1_t64": (3, 2, 2, 576, 64, 64, [(1, 5), (2, 3)], 4),
 }
 
 
 @pytest.mark.parametrize("name", list(CASES))
 def test_host_prefill_equals_device_path(T, oracle_mod, name):
-    B, Hq, Hkv, S, D, Tb, pol = CASES[name]
+    B, Hq, Hkv, S, D, Tb, pol, slots = CASES[name]
     hi = np.array([p[0] for p in pol], np.int32)
     keep = np.array([p[1] for p in pol], np.int32)
     seed = sum(map(ord, name))
@@ -59,7 +60,7 @@ def test_host_prefill_equals_device_path(T, oracle_mod, name):
     hQ, hK, hV = (t.pin_memory() for t in (Q, K, V))
     hO = torch.full((B, Hq, S, D), float("nan"), dtype=torch.bfloat16).pin_memory()
     hL = torch.full((B, Hq, S), float("nan"), dtype=torch.float32).pin_memory()
-    run = T.HostPrefill(B, Hq, Hkv, S, D, Tb)
+    run = T.HostPrefill(B, Hq, Hkv, S, D, Tb, slots=slots)
     for _ in range(2):   # twice: the second call reuses the staging slots and workspace
         run(hQ, hK, hV, cache, hi, keep, hO, hL)
     torch.cuda.current_stream().synchronize()
