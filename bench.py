@@ -358,7 +358,9 @@ def prefill_leg(tria, w, args, flush, stream, clocks=None, e2e=True):
            "work": prefill_work(w, hi, keep, tria),
            "decode_bytes": decode_bytes(w.B, w.Hq, w.Hkv, w.D, w.T, kv_len, hi, keep),
            "codec_bytes": 2 * (K.numel() * 2) + 2 * (K.numel() + K.numel() // 2) + 4 * 4 * K.numel() // w.D,
-           "launches_per_step": 2 + 2 + 1 + 2}
+           # cache write (one launch for K and V), Q codec + preparation, fused kernel,
+           # decode + merge
+           "launches_per_step": 1 + 2 + 1 + 2}
     if e2e:
         # The user's call from host memory: tria_prefill_host writes the cache and runs the
         # prefill group by group, its copies in and out overlapping the kernels; then the
