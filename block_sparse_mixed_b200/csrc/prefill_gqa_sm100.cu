@@ -55,6 +55,35 @@ constexpr int kUnitRing = 16;
 constexpr int kLastLoad = 1 << 8;       // info.z flags next to the plane
 constexpr int kLastOfPlane = 1 << 9;    // the tile's last load of this plane: its QK frees the Q buffer
 
+// Output rows of one warp, coalesced. Lane l holds NC 16-byte chunks (chunk[c], 8
+// bf16 values each) of row l of the warp's 32 rows, for the same columns in every
+// row; row l goes to dst0 + l * row_stride (bytes), lanes whose row is not valid hold
+// nothing to write. Written straight from the lanes, every store instruction would
+// touch 32 rows; instead the warp passes the chunks through `scratch` (32 * NC * 16
+// bytes of shared memory that only this warp uses) so that each store instruction
+// writes 32 / NC whole row segments of NC * 16 bytes. Chunk c of row l is kept at
+// position c ^ ((l / (8 / NC)) % NC) of its row, so that neither the writes of one
+// chunk by all lanes nor the reads of 32 / NC consecutive rows meet a bank twice
+// within a 128-byte wavefront.
+template <int NC>
+__device__ __forceinline__ void store_rows(const uint4 (&chunk)[NC], bool valid, uint8_t* scratch, uint8_t* dst0,
+                                           int64_t row_stride, int lane) {
+  static_assert(NC == 4 || NC == 8, "row segment of 64 or 128 bytes");
+  constexpr int kRowsPerStore = 32 / NC;
+  auto pos = [](int l, int c) { return l * NC * 16 + ((c ^ ((l / (8 / NC)) % NC)) << 4); };
+#pragma unroll
+  for (int c = 0; c < NC; ++c) *reinterpret_cast<uint4*>(scratch + pos(lane, c)) = chunk[c];
+  const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < NC; ++i) {
+    const int l = i * kRowsPerStore + lane / NC, c = lane % NC;
+    const uint4 v = *reinterpret_cast<const uint4*>(scratch + pos(l, c));
+    if ((vmask >> l) & 1u) *reinterpret_cast<uint4*>(dst0 + l * row_stride + c * 16) = v;
+  }
+  __syncwarp();   // the scratch is free again for this warp's next writes
+}
+
 // S slot of head p: columns 128 p; O accumulator of head p: 256 + 128 p.
 __host__ __device__ constexpr uint32_t s_col(int p) { return 128u * static_cast<uint32_t>(p); }
 __host__ __device__ constexpr uint32_t o_col(int p) { return 256u + 128u * static_cast<uint32_t>(p); }
@@ -582,17 +611,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < HC / 32; ++c) tmem_ld32(my_o + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&o[32 * c]));
       tmem_wait_ld();
-      if (valid) {
-        uint4* dst = reinterpret_cast<uint4*>(a.O + qrow * D + half * HC);
+      {
+        uint4 ch[HC / 8];
 #pragma unroll
         for (int k = 0; k < HC / 8; ++k) {
           uint32_t wv[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e)
             wv[e] = bf16x2(__uint_as_float(o[8 * k + 2 * e]) * inv_l, __uint_as_float(o[8 * k + 2 * e + 1]) * inv_l);
-          dst[k] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          ch[k] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
         }
-        if (half == 0) a.LSE[qrow] = (m_run + log2f(l_tot)) * 0.69314718055994531f;
+        // through the warp's own 32 rows of the head's P sub-tile: the head's last P.V
+        // has completed, so the tensor core reads nothing there any more
+        store_rows<HC / 8>(ch, valid, sP(pair) + half * C::kPSub + sub * 32 * 128,
+                           reinterpret_cast<uint8_t*>(a.O + (qrow - lane) * D + half * HC), D * 2, lane);
+        if (valid && half == 0) a.LSE[qrow] = (m_run + log2f(l_tot)) * 0.69314718055994531f;
       }
       // both halves have read the sums before the next tile's exchange overwrites them;
       // O_p is read before this pair's next P (and so the next P.V) is written

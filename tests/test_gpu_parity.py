@@ -163,6 +163,11 @@ PREFILL_CASES = {
     "protected_only": (1, 2, 2, 640, 128, 64, [(0, 0), (0, 1)]),
     "dense_int8": (1, 2, 1, 512, 128, 128, [(4, 4), (9, 9)]),
     "all_int4_band": (1, 2, 1, 512, 128, 64, [(0, 20), (1, 20)]),
+    # head pairs with equal boundaries: the GQA-shared kernel (its staged O stores),
+    # with a last tile of one query block at T = 64
+    "gqa_shared_ragged_t64": (2, 4, 2, 576, 128, 64, [(1, 2), (1, 2), (3, 9), (3, 9)]),
+    "gqa_shared_d64_t64": (1, 4, 1, 704, 64, 64, [(2, 5), (2, 5), (0, 3), (0, 3)]),
+    "gqa_shared_d64_t128": (1, 4, 2, 896, 64, 128, [(1, 4), (1, 4), (2, 7), (2, 7)]),
 }
 
 
