@@ -515,8 +515,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = qb < u.nq;
       const int ir = u.i0 + qb;
       const int64_t qrow = (static_cast<int64_t>(u.b) * a.Hq + u.hq) * a.S + static_cast<int64_t>(ir) * T + rl;
-      const float a8 = valid ? a.q8s[qrow] * a.qk_log2 : 0.0f;
-      const float a4 = valid ? a.q4s[qrow] * a.qk_log2 : 0.0f;
+      // the row's query scales, taken times log2(e) / sqrt(D) only where a load's plane
+      // picks one: nothing before the first load's waits consumes the two reads
+      const float q8s = valid ? a.q8s[qrow] : 0.0f;
+      const float q4s = valid ? a.q4s[qrow] : 0.0f;
       const int hi = a.hi[u.hq], keep = a.keep[u.hq];
       float m_run = -INFINITY, l_run = 0.0f;     // m_run: shared by both halves of the pair
       // this tile's loads are g0 .. g0 + n - 1 in the CTA's order; the pair takes
@@ -538,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // uniform over the warp (its 32 rows are in one query block)
         const int act = (valid && jh >= 0) ? tile_action(ir, jh, hi, keep) : ACT_NONE;
         const bool active = act == plane;
-        const float alpha = plane == 8 ? a8 : a4;
+        const float alpha = (plane == 8 ? q8s : q4s) * a.qk_log2;
         const int kmax = (jh == ir) ? rl - koff : TH;   // my keys [0, kmax] are visible
         float* xb = xmax + pair * 256;
         // Both halves exchange their maxima on every load (an inactive half offers
