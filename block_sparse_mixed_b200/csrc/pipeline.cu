@@ -8,7 +8,12 @@
 // cache rows, its query heads and its outputs are its own), so group g's kernels run
 // while group g + 1's inputs are copied in and group g - 1's outputs are copied out,
 // through two to four staging slots in device memory (as many as the caller's
-// staging buffer holds).
+// staging buffer holds). The copies in set the pace; what runs after the last of them
+// (the last unit's kernels and its copy out) is the pipeline's tail, so the last group
+// is taken as two units of G / 2 query heads when G is a multiple of 4 (head pairs
+// with the same boundaries stay together, so every head is computed by the same
+// kernel as in a whole-group unit): the first writes the group's cache rows, the
+// second only copies its queries in.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -108,8 +113,10 @@ int tria_prefill_host(const void* hQ, const void* hK, const void* hV, const tria
   const cudaStream_t so = static_cast<cudaStream_t>(copy_out_stream);
   const int G = d.Hq / d.Hkv;
   const int groups = d.B * d.Hkv;
-  const size_t qbytes = static_cast<size_t>(G) * d.S * d.D * 2, kvbytes = static_cast<size_t>(d.S) * d.D * 2;
-  const size_t obytes = qbytes, lbytes = static_cast<size_t>(G) * d.S * 4;
+  const bool split_last = G % 4 == 0;
+  const int units = groups + (split_last ? 1 : 0);
+  const size_t kvbytes = static_cast<size_t>(d.S) * d.D * 2;
+  const size_t head_q = static_cast<size_t>(d.S) * d.D * 2, head_l = static_cast<size_t>(d.S) * 4;   // per query head
   uint8_t* st = static_cast<uint8_t*>(staging);
   auto q_of = [&](int s) { return st + s * sz.slot; };
   auto k_of = [&](int s) { return q_of(s) + sz.q; };
@@ -142,38 +149,50 @@ int tria_prefill_host(const void* hQ, const void* hK, const void* hV, const tria
   if (status == TRIA_OK && ok(cudaEventRecord(start, sc)) && ok(cudaStreamWaitEvent(si, start, 0)))
     ok(cudaStreamWaitEvent(so, start, 0));
 
-  for (int gi = 0; gi < groups && status == TRIA_OK; ++gi) {
-    const int s = gi % slots;
+  for (int ui = 0; ui < units && status == TRIA_OK; ++ui) {
+    const int s = ui % slots;
+    // unit ui: group gi, query heads [h0, h0 + nh) of it; the group's first unit writes its cache rows
+    const bool second_half = split_last && ui == units - 1;
+    const int gi = second_half ? groups - 1 : ui;
+    const int nh = split_last && gi == groups - 1 ? G / 2 : G;
+    const int h0 = second_half ? G / 2 : 0;
+    const bool write_cache = h0 == 0;
     const int b = gi / d.Hkv, kvh = gi % d.Hkv;
-    const size_t qrow0 = static_cast<size_t>(b) * d.Hq + static_cast<size_t>(kvh) * G;   // first query head row
-    // inputs of group gi into slot s, once group gi - slots has consumed it
-    if (gi >= slots && !ok(cudaStreamWaitEvent(si, in_free(s), 0))) break;
-    if (!ok(cudaMemcpyAsync(k_of(s), static_cast<const uint8_t*>(hK) + gi * kvbytes, kvbytes, cudaMemcpyHostToDevice, si)))
-      break;
-    if (!ok(cudaMemcpyAsync(v_of(s), static_cast<const uint8_t*>(hV) + gi * kvbytes, kvbytes, cudaMemcpyHostToDevice, si)))
-      break;
-    if (!ok(cudaMemcpyAsync(q_of(s), static_cast<const uint8_t*>(hQ) + qrow0 * d.S * d.D * 2, qbytes,
+    const size_t qrow0 = static_cast<size_t>(b) * d.Hq + static_cast<size_t>(kvh) * G + h0;   // first query head row
+    tria_dims ud = gd;
+    ud.Hq = nh;
+    // inputs of unit ui into slot s, once unit ui - slots has consumed it
+    if (ui >= slots && !ok(cudaStreamWaitEvent(si, in_free(s), 0))) break;
+    if (write_cache) {
+      if (!ok(cudaMemcpyAsync(k_of(s), static_cast<const uint8_t*>(hK) + gi * kvbytes, kvbytes, cudaMemcpyHostToDevice,
+                              si)))
+        break;
+      if (!ok(cudaMemcpyAsync(v_of(s), static_cast<const uint8_t*>(hV) + gi * kvbytes, kvbytes, cudaMemcpyHostToDevice,
+                              si)))
+        break;
+    }
+    if (!ok(cudaMemcpyAsync(q_of(s), static_cast<const uint8_t*>(hQ) + qrow0 * head_q, nh * head_q,
                             cudaMemcpyHostToDevice, si)))
       break;
     if (!ok(cudaEventRecord(in_ready(s), si))) break;
-    // kernels of group gi: cache write, preparation, fused prefill into slot s's outputs
-    // (once group gi - slots' outputs have been copied out of it)
+    // kernels of unit ui: cache write (the group's first unit), preparation, fused
+    // prefill into slot s's outputs (once unit ui - slots' outputs have been copied out of it)
     if (!ok(cudaStreamWaitEvent(sc, in_ready(s), 0))) break;
-    if (gi >= slots && !ok(cudaStreamWaitEvent(sc, out_free(s), 0))) break;
+    if (ui >= slots && !ok(cudaStreamWaitEvent(sc, out_free(s), 0))) break;
     const tria_kv_cache gc = group_cache(*cache, gi);
-    if (!ok_t(tria_quantize_kv(k_of(s), v_of(s), d.S, 0, &gc, sc))) break;
-    if (!ok_t(tria_prefill_prepare(q_of(s), &gc, &gd, workspace, workspace_bytes, sc))) break;
+    if (write_cache && !ok_t(tria_quantize_kv(k_of(s), v_of(s), d.S, 0, &gc, sc))) break;
+    if (!ok_t(tria_prefill_prepare(q_of(s), &gc, &ud, workspace, workspace_bytes, sc))) break;
     if (!ok(cudaEventRecord(in_free(s), sc))) break;
-    if (!ok_t(tria_prefill_attend(&gc, &gd, hi + kvh * G, keep + kvh * G, o_of(s), l_of(s), workspace,
+    if (!ok_t(tria_prefill_attend(&gc, &ud, hi + kvh * G + h0, keep + kvh * G + h0, o_of(s), l_of(s), workspace,
                                   workspace_bytes, sc)))
       break;
     if (!ok(cudaEventRecord(out_ready(s), sc))) break;
-    // outputs of group gi to the host
+    // outputs of unit ui to the host
     if (!ok(cudaStreamWaitEvent(so, out_ready(s), 0))) break;
-    if (!ok(cudaMemcpyAsync(static_cast<uint8_t*>(hO) + qrow0 * d.S * d.D * 2, o_of(s), obytes, cudaMemcpyDeviceToHost,
+    if (!ok(cudaMemcpyAsync(static_cast<uint8_t*>(hO) + qrow0 * head_q, o_of(s), nh * head_q, cudaMemcpyDeviceToHost,
                             so)))
       break;
-    if (!ok(cudaMemcpyAsync(hLSE + qrow0 * d.S, l_of(s), lbytes, cudaMemcpyDeviceToHost, so))) break;
+    if (!ok(cudaMemcpyAsync(hLSE + qrow0 * d.S, l_of(s), nh * head_l, cudaMemcpyDeviceToHost, so))) break;
     if (!ok(cudaEventRecord(out_free(s), so))) break;
   }
   // `stream` completes after the last copy out (and after any copy in, on an early stop)

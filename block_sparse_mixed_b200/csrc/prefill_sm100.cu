@@ -656,7 +656,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool use0 = l0 > 0.0f, use1 = l1 > 0.0f;
       const float w0 = use0 ? fast_exp2(m0 - m_all) : 0.0f;
       const float w1 = use1 ? fast_exp2(m1 - m_all) : 0.0f;
-      const float l_tot = l0 * w0 + l1 * w1;
+      // The two accumulators hold the tile's loads of even and odd position in either
+      // order (which one takes the first load depends on the CTA's running load count,
+      // so on the tiles it drew before): both products are rounded before the one
+      // commutative add, here and for O, so the bits do not depend on that order
+      // (a contracted fma(l0, w0, l1 * w1) would round only one of them).
+      const float l_tot = __fmul_rn(l0, w0) + __fmul_rn(l1, w1);
       const float inv_l = valid ? 1.0f / l_tot : 0.0f;
       const float f0 = w0 * inv_l, f1 = w1 * inv_l;
       // this thread writes output columns [quarter * D/4, (quarter+1) * D/4)
@@ -679,9 +684,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int i0 = 8 * k + 2 * e;
-            const float v0 = (use0 ? __uint_as_float(o0[i0]) * f0 : 0.0f) + (use1 ? __uint_as_float(o1[i0]) * f1 : 0.0f);
-            const float v1 =
-                (use0 ? __uint_as_float(o0[i0 + 1]) * f0 : 0.0f) + (use1 ? __uint_as_float(o1[i0 + 1]) * f1 : 0.0f);
+            const float v0 = (use0 ? __fmul_rn(__uint_as_float(o0[i0]), f0) : 0.0f) +
+                             (use1 ? __fmul_rn(__uint_as_float(o1[i0]), f1) : 0.0f);
+            const float v1 = (use0 ? __fmul_rn(__uint_as_float(o0[i0 + 1]), f0) : 0.0f) +
+                             (use1 ? __fmul_rn(__uint_as_float(o1[i0 + 1]), f1) : 0.0f);
             wv[e] = bf16x2(v0, v1);
           }
           dst[k] = make_uint4(wv[0], wv[1], wv[2], wv[3]);

@@ -215,7 +215,9 @@ int tria_prefill_gqa(int enable);
  * with the kernels. The work is split by (batch, KV head) group: group g's K, V and
  * its Hq/Hkv query heads' Q are copied in on copy_in_stream while group g - 1's
  * kernels run on `stream` and group g - 2's O and LSE are copied out on
- * copy_out_stream, through the slots of `staging`.
+ * copy_out_stream, through the slots of `staging`. When Hq/Hkv is a multiple of 4
+ * the last group goes as two units of half its query heads (the first also writes
+ * the group's cache rows), which halves the work left after the last copy in.
  *   hQ, hK, hV    host bf16, [B,Hq,S,D] and [B,Hkv,S,D]; page-locked memory lets the
  *                 copies overlap (pageable memory works, serialised by the runtime).
  *   hO, hLSE      host bf16 [B,Hq,S,D] and fp32 [B,Hq,S], written by the call.

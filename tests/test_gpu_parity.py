@@ -210,6 +210,31 @@ def test_prefill_llama_workload_sampled_rows(T, oracle_mod):
     compare_lse(L.reshape(-1).cpu()[idx], L_ref, "llama sampled")
 
 
+@pytest.mark.parametrize("name", ["llama_prefill", "llama_prefill_gqa"])
+def test_prefill_is_deterministic(T, name):
+    """Two calls on the same cache give the same bits. The per-head kernel splits a
+    tile's loads between two accumulators by the parity of the CTA's running load
+    count, which depends on which tiles the CTA drew from the tile counter; the two
+    partial results are merged commutatively, so the bits must not depend on it."""
+    w = W.WORKLOADS[name]
+    Q, K, V = W.prefill_inputs(w)
+    hi, keep = W.policy(w)
+    cache = T.CompressedKVCache(w.B, w.Hkv, w.D, w.T, w.S)
+    T.tria_quantize_kv(K.cuda(), V.cuda(), cache)
+    Qd = Q.cuda()
+    outs = []
+    for _ in range(3):
+        O = torch.full_like(Qd, float("nan"))
+        L = torch.full((w.B, w.Hq, w.S), float("nan"), dtype=torch.float32, device="cuda")
+        T.tria_prefill(Qd, cache, hi, keep, O=O, LSE=L)
+        outs.append((O, L))
+    torch.cuda.synchronize()
+    for O, L in outs[1:]:
+        assert torch.equal(O.view(torch.int16), outs[0][0].view(torch.int16)), name
+        assert torch.equal(L.view(torch.int32), outs[0][1].view(torch.int32)), name
+    assert not torch.isnan(outs[0][0].float()).any() and not torch.isnan(outs[0][1]).any()
+
+
 @pytest.mark.parametrize("Tb", [64, 128])
 def test_prefill_many_short_tiles_sampled_rows(T, oracle_mod, Tb):
     """Tiles of one to three loads each, about 17 per CTA: each CTA runs through
@@ -329,6 +354,23 @@ def test_decode_workload_four_sequences(T, oracle_mod):
     O_ref, L_ref = oracle_mod.decode(q, K, V, w.T, kv, hi, keep)
     compare_o(O, O_ref, "decode workload")
     compare_lse(L, L_ref, "decode workload")
+
+
+def test_decode_is_deterministic(T):
+    """Two decode calls on the same cache give the same bits, whichever CTA draws which
+    work item: every (item, warp) partial has its own slot and the merge adds them in
+    slot order."""
+    w = W.scaled(W.WORKLOADS["decode"], B=16)
+    q, K, V, kv = W.decode_inputs(w)
+    hi, keep = W.policy(w)
+    cache = T.CompressedKVCache(w.B, w.Hkv, w.D, w.T, K.shape[2])
+    T.tria_quantize_kv(K.cuda(), V.cuda(), cache)
+    qd = q.cuda()
+    outs = [T.tria_decode(qd, cache, kv, hi, keep) for _ in range(3)]
+    torch.cuda.synchronize()
+    for O, L in outs[1:]:
+        assert torch.equal(O.view(torch.int16), outs[0][0].view(torch.int16))
+        assert torch.equal(L.view(torch.int32), outs[0][1].view(torch.int32))
 
 
 def test_decode_equals_last_prefill_row(T):
