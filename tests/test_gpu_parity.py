@@ -210,13 +210,14 @@ def test_prefill_llama_workload_sampled_rows(T, oracle_mod):
     compare_lse(L.reshape(-1).cpu()[idx], L_ref, "llama sampled")
 
 
-@pytest.mark.parametrize("name", ["llama_prefill", "llama_prefill_gqa"])
+@pytest.mark.parametrize("name", ["llama_prefill", "llama_prefill_gqa", "long_prefill_b1"])
 def test_prefill_is_deterministic(T, name):
     """Two calls on the same cache give the same bits. The per-head kernel splits a
     tile's loads between two accumulators by the parity of the CTA's running load
     count, which depends on which tiles the CTA drew from the tile counter; the two
-    partial results are merged commutatively, so the bits must not depend on it."""
-    w = W.WORKLOADS[name]
+    partial results are merged commutatively, so the bits must not depend on it.
+    long_prefill_b1: one sequence of the 32,768-token workload (T = 128, 55 tiles per CTA)."""
+    w = W.scaled(W.WORKLOADS["long_prefill"], B=1) if name == "long_prefill_b1" else W.WORKLOADS[name]
     Q, K, V = W.prefill_inputs(w)
     hi, keep = W.policy(w)
     cache = T.CompressedKVCache(w.B, w.Hkv, w.D, w.T, w.S)
