@@ -560,10 +560,18 @@ int tria_decode(const void* q, const tria_kv_cache* cache, const int32_t* kv_len
     for (int g = 0; g < groups; ++g) n += (nkept[g] + b - 1) / b;
     return n;
   };
-  // sum over groups of ceil(n_g / bps) <= total / bps + groups
-  if (L.max_items > groups)
-    bps = std::max<int64_t>(bps, (total + (L.max_items - groups) - 1) / (L.max_items - groups));
-  while (count_items(bps) > L.max_items) ++bps;
+  // the smallest split size from there whose items fit the workspace's partial slots
+  // (the item count falls as the split size grows; at the largest group's size it is
+  // one item per group, within the slots)
+  if (count_items(bps) > L.max_items) {
+    int lo = bps, hi = 1;
+    for (int g = 0; g < groups; ++g) hi = std::max(hi, nkept[g]);
+    while (lo < hi) {
+      const int mid = lo + (hi - lo) / 2;
+      if (count_items(mid) <= L.max_items) hi = mid; else lo = mid + 1;
+    }
+    bps = lo;
+  }
 
   DecodeArgs a{};
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.G = G; a.D = D; a.T = T;
