@@ -21,6 +21,7 @@ namespace tria {
 namespace {
 
 constexpr int kRowsPerTile = 128;   // query rows of a fused-prefill tile
+constexpr int kCostLevels = 8192;   // levels of the decode's first-split cost estimate (in blocks)
 
 // Whether the fused prefill may use the GQA-shared kernel (tria_prefill_gqa).
 std::atomic<bool> g_prefill_gqa{true};
@@ -596,6 +597,28 @@ int tria_decode(const void* q, const tria_kv_cache* cache, const int32_t* kv_len
   }
   a.split_start[groups] = items;
   a.n_items = items;
+  // The groups' first splits go last, the costlier first (a counting sort): a split's
+  // blocks, plus the diagonal band's 8-bit blocks (counted twice, the largest band of
+  // the group's heads) when the group has a single split.
+  {
+    std::vector<int> cost(groups), count(kCostLevels, 0);
+    for (int g = 0; g < groups; ++g) {
+      const int n = a.split_start[g + 1] - a.split_start[g];
+      const int first = nkept[g] - (n - 1) * bps;
+      int band = 0;
+      if (n == 1)
+        for (int h = 0; h < G; ++h) band = std::max(band, hi[(g % Hkv) * G + h]);
+      cost[g] = static_cast<int>(std::min<int64_t>(static_cast<int64_t>(first) + band, kCostLevels - 1));
+      ++count[cost[g]];
+    }
+    int at = 0;   // descending cost: start offsets from the top
+    for (int c = static_cast<int>(count.size()) - 1; c >= 0; --c) {
+      const int n = count[c];
+      count[c] = at;
+      at += n;
+    }
+    for (int g = 0; g < groups; ++g) a.first_order[count[cost[g]]++] = static_cast<int16_t>(g);
+  }
 
   DecodeMaps maps;
   const uint64_t rows = static_cast<uint64_t>(a.ci.rows(B));   // below 2^31 (check_cache)

@@ -137,6 +137,7 @@ struct DecodeArgs {
   int keep[kMaxHeads];
   int kv_len[kMaxBatch];
   int split_start[kMaxGroups + 1];     // first work item of each group (groups = B*Hkv)
+  int16_t first_order[kMaxGroups];     // the group of each item of the last phase (see item_range)
 };
 
 cudaError_t launch_quant_rows(const QuantArgs& a, int D, cudaStream_t stream);
