@@ -202,6 +202,73 @@ DecodeLayout decode_layout(int B, int Hq, int Hkv, int D) {
   return L;
 }
 
+// The decode's work plan (host side). nkept[g]: kept key blocks of group g = b * Hkv +
+// kvh at its query position, the union over its G heads (block 0, then every block from
+// the first one the widest band keeps to the diagonal). The split size bps asks for
+// about six items per SM (at least 4 blocks), enlarged to the smallest size whose items
+// fit max_items partial slots; split_start[g] is group g's first item and slot
+// (ceil(nkept / bps) items each), and first_order lists the groups' first splits, the
+// last phase of the launch, costliest first (a counting sort on the split's blocks plus,
+// for a group of a single split, its widest 8-bit band once more). Returns the number
+// of items.
+int decode_plan(int B, int Hkv, int G, int T, const int32_t* kv_len, const int32_t* hi, const int32_t* keep, int sms,
+                int max_items, int* bps_out, int* nkept, int* split_start, int16_t* first_order) {
+  const int groups = B * Hkv;
+  int64_t total = 0;
+  for (int b = 0; b < B; ++b)
+    for (int k = 0; k < Hkv; ++k) {
+      const int ib = (kv_len[b] - 1) / T;
+      int mk = 0;
+      for (int h = 0; h < G; ++h) mk = std::max(mk, keep[k * G + h]);
+      const int jb = first_band_block(ib, mk);
+      nkept[b * Hkv + k] = ib == 0 ? 1 : 1 + (ib - jb + 1);
+      total += nkept[b * Hkv + k];
+    }
+  const int64_t target_items = static_cast<int64_t>(sms) * 6;
+  int bps = static_cast<int>(std::max<int64_t>(4, (total + target_items - 1) / target_items));
+  auto count_items = [&](int b) {
+    int64_t n = 0;
+    for (int g = 0; g < groups; ++g) n += (nkept[g] + b - 1) / b;
+    return n;
+  };
+  // the item count falls as the split size grows; at the largest group's size it is one
+  // item per group, within the slots
+  if (count_items(bps) > max_items) {
+    int lo = bps, top = 1;
+    for (int g = 0; g < groups; ++g) top = std::max(top, nkept[g]);
+    while (lo < top) {
+      const int mid = lo + (top - lo) / 2;
+      if (count_items(mid) <= max_items) top = mid; else lo = mid + 1;
+    }
+    bps = lo;
+  }
+  int items = 0;
+  for (int g = 0; g < groups; ++g) {
+    split_start[g] = items;
+    items += (nkept[g] + bps - 1) / bps;
+  }
+  split_start[groups] = items;
+  std::vector<int> cost(groups), count(kCostLevels, 0);
+  for (int g = 0; g < groups; ++g) {
+    const int n = split_start[g + 1] - split_start[g];
+    const int first = nkept[g] - (n - 1) * bps;
+    int band = 0;
+    if (n == 1)
+      for (int h = 0; h < G; ++h) band = std::max(band, hi[(g % Hkv) * G + h]);
+    cost[g] = static_cast<int>(std::min<int64_t>(static_cast<int64_t>(first) + band, kCostLevels - 1));
+    ++count[cost[g]];
+  }
+  int at = 0;   // descending cost: start offsets from the top
+  for (int c = kCostLevels - 1; c >= 0; --c) {
+    const int n = count[c];
+    count[c] = at;
+    at += n;
+  }
+  for (int g = 0; g < groups; ++g) first_order[count[cost[g]]++] = static_cast<int16_t>(g);
+  *bps_out = bps;
+  return items;
+}
+
 }  // namespace
 }  // namespace tria
 
@@ -342,6 +409,36 @@ int tria_count_tiles(int nb, int hi, int keep, int64_t* out) {
       const int a = tile_action(i, j, hi, keep);
       if (a == ACT_INT8) ++out[0]; else if (a == ACT_INT4) ++out[1]; else if (a == ACT_SKIP) ++out[2];
     }
+  return TRIA_OK;
+}
+
+int tria_decode_plan(int B, int Hq, int Hkv, int T, int capacity, const int32_t* kv_len, const int32_t* hi,
+                     const int32_t* keep, int num_sms, int32_t* split_start, int32_t* first_order, int32_t* nkept,
+                     int32_t* blocks_per_split, int32_t* n_items) {
+  if (B < 1 || Hkv < 1 || Hq < 1 || Hq % Hkv != 0 || (T != 64 && T != 128) || capacity < 1 || capacity % T != 0 ||
+      num_sms < 1 || kv_len == nullptr || split_start == nullptr || first_order == nullptr || nkept == nullptr ||
+      blocks_per_split == nullptr || n_items == nullptr)
+    return TRIA_ERR_INVALID_ARG;
+  if (Hq > kMaxHeads || Hq / Hkv > 16 || B > kMaxBatch || static_cast<int64_t>(B) * Hkv > kMaxGroups)
+    return TRIA_ERR_UNSUPPORTED;
+  int s = check_policy(hi, keep, Hq);
+  if (s != TRIA_OK) return s;
+  for (int b = 0; b < B; ++b)
+    if (kv_len[b] < 1 || kv_len[b] > capacity) return TRIA_ERR_INVALID_ARG;
+  const int groups = B * Hkv;
+  std::vector<int> nk(groups), ss(groups + 1);
+  std::vector<int16_t> fo(groups);
+  int bps = 0;
+  const int items = decode_plan(B, Hkv, Hq / Hkv, T, kv_len, hi, keep, num_sms, decode_max_items(groups), &bps,
+                                nk.data(), ss.data(), fo.data());
+  for (int g = 0; g < groups; ++g) {
+    nkept[g] = nk[g];
+    split_start[g] = ss[g];
+    first_order[g] = fo[g];
+  }
+  split_start[groups] = ss[groups];
+  *blocks_per_split = bps;
+  *n_items = items;
   return TRIA_OK;
 }
 
@@ -540,41 +637,13 @@ int tria_decode(const void* q, const tria_kv_cache* cache, const int32_t* kv_len
   const int G = Hq / Hkv;
   const int groups = B * Hkv;
 
-  // kept key blocks per group (union over the group's heads), then the split size
+  // the work plan: kept blocks per group, split size, each group's first item, the
+  // order of the groups' first splits
   std::vector<int> nkept(groups);
-  int64_t total = 0;
-  for (int b = 0; b < B; ++b)
-    for (int k = 0; k < Hkv; ++k) {
-      const int ib = (kv_len[b] - 1) / T;
-      int mk = 0;
-      for (int h = 0; h < G; ++h) mk = std::max(mk, keep[k * G + h]);
-      const int jb = first_band_block(ib, mk);
-      nkept[b * Hkv + k] = ib == 0 ? 1 : 1 + (ib - jb + 1);
-      total += nkept[b * Hkv + k];
-    }
-  // about six items per SM; items of one group are consecutive runs of its kept blocks
-  const int64_t target_items = static_cast<int64_t>(dev.sms) * 6;
-  // (at least 4 blocks: small problems are bound by latency, and fewer partials merge faster)
-  int bps = static_cast<int>(std::max<int64_t>(4, (total + target_items - 1) / target_items));
-  auto count_items = [&](int b) {
-    int64_t n = 0;
-    for (int g = 0; g < groups; ++g) n += (nkept[g] + b - 1) / b;
-    return n;
-  };
-  // the smallest split size from there whose items fit the workspace's partial slots
-  // (the item count falls as the split size grows; at the largest group's size it is
-  // one item per group, within the slots)
-  if (count_items(bps) > L.max_items) {
-    int lo = bps, hi = 1;
-    for (int g = 0; g < groups; ++g) hi = std::max(hi, nkept[g]);
-    while (lo < hi) {
-      const int mid = lo + (hi - lo) / 2;
-      if (count_items(mid) <= L.max_items) hi = mid; else lo = mid + 1;
-    }
-    bps = lo;
-  }
-
+  int bps = 0;
   DecodeArgs a{};
+  const int items = decode_plan(B, Hkv, G, T, kv_len, hi, keep, dev.sms, L.max_items, &bps, nkept.data(),
+                                a.split_start, a.first_order);
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.G = G; a.D = D; a.T = T;
   a.ci = cache_index(*cache);
   a.blocks_per_split = bps;
@@ -590,35 +659,7 @@ int tria_decode(const void* q, const tria_kv_cache* cache, const int32_t* kv_len
   a.n_groups = groups;
   for (int h = 0; h < Hq; ++h) { a.hi[h] = hi[h]; a.keep[h] = keep[h]; }
   for (int b = 0; b < B; ++b) a.kv_len[b] = kv_len[b];
-  int items = 0;
-  for (int g = 0; g < groups; ++g) {
-    a.split_start[g] = items;
-    items += (nkept[g] + bps - 1) / bps;
-  }
-  a.split_start[groups] = items;
   a.n_items = items;
-  // The groups' first splits go last, the costlier first (a counting sort): a split's
-  // blocks, plus the diagonal band's 8-bit blocks (counted twice, the largest band of
-  // the group's heads) when the group has a single split.
-  {
-    std::vector<int> cost(groups), count(kCostLevels, 0);
-    for (int g = 0; g < groups; ++g) {
-      const int n = a.split_start[g + 1] - a.split_start[g];
-      const int first = nkept[g] - (n - 1) * bps;
-      int band = 0;
-      if (n == 1)
-        for (int h = 0; h < G; ++h) band = std::max(band, hi[(g % Hkv) * G + h]);
-      cost[g] = static_cast<int>(std::min<int64_t>(static_cast<int64_t>(first) + band, kCostLevels - 1));
-      ++count[cost[g]];
-    }
-    int at = 0;   // descending cost: start offsets from the top
-    for (int c = static_cast<int>(count.size()) - 1; c >= 0; --c) {
-      const int n = count[c];
-      count[c] = at;
-      at += n;
-    }
-    for (int g = 0; g < groups; ++g) a.first_order[count[cost[g]]++] = static_cast<int16_t>(g);
-  }
 
   DecodeMaps maps;
   const uint64_t rows = static_cast<uint64_t>(a.ci.rows(B));   // below 2^31 (check_cache)

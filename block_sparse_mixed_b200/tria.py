@@ -73,6 +73,8 @@ def lib():
         L.tria_count_tiles.restype = I
         L.tria_prefill_load_plan.argtypes = [I, I, I, I, P, I64, P]
         L.tria_prefill_load_plan.restype = I
+        L.tria_decode_plan.argtypes = [I, I, I, I, I, P, P, P, I, P, P, P, P, P]
+        L.tria_decode_plan.restype = I
         L.tria_prefill_workspace_bytes.argtypes = [ctypes.POINTER(tria_dims)]
         L.tria_prefill_workspace_bytes.restype = SZ
         L.tria_prefill.argtypes = [P, ctypes.POINTER(tria_kv_cache), ctypes.POINTER(tria_dims), P, P, P, P, P,
@@ -223,6 +225,21 @@ def tria_prefill_load_plan(nb: int, T: int, hi: int, keep: int) -> np.ndarray:
     _check("tria_prefill_load_plan", lib().tria_prefill_load_plan(nb, T, hi, keep, out.ctypes.data_as(ctypes.c_void_p),
                                                                   n.value, ctypes.byref(n)))
     return out
+
+
+def tria_decode_plan(B: int, Hq: int, Hkv: int, T: int, capacity: int, kv_len, hi, keep, num_sms: int) -> dict:
+    """The decode's work plan: {'nkept', 'split_start', 'first_order', 'blocks_per_split', 'n_items'}."""
+    groups = B * Hkv
+    ss = np.zeros(groups + 1, np.int32)
+    fo = np.zeros(groups, np.int32)
+    nk = np.zeros(groups, np.int32)
+    bps, n = ctypes.c_int32(0), ctypes.c_int32(0)
+    P = ctypes.c_void_p
+    kv_a, hi_a, keep_a = _host_i32(kv_len), _host_i32(hi), _host_i32(keep)
+    _check("tria_decode_plan", lib().tria_decode_plan(
+        B, Hq, Hkv, T, capacity, kv_a.ctypes.data_as(P), hi_a.ctypes.data_as(P), keep_a.ctypes.data_as(P), num_sms,
+        ss.ctypes.data_as(P), fo.ctypes.data_as(P), nk.ctypes.data_as(P), ctypes.byref(bps), ctypes.byref(n)))
+    return {"nkept": nk, "split_start": ss, "first_order": fo, "blocks_per_split": bps.value, "n_items": n.value}
 
 
 def tria_prefill_workspace_bytes(B, Hq, Hkv, S, D, T) -> int:

@@ -258,6 +258,24 @@ int tria_prefill_attend(const tria_kv_cache* cache, const tria_dims* dims, const
                         const int32_t* keep, void* O, float* LSE, void* workspace, size_t workspace_bytes,
                         void* stream);
 
+/* The work plan tria_decode launches with (host-only helper; the decode kernel's
+ * producer maps each work item to a group and a run of its kept blocks from it). The
+ * kept blocks are the union over a group's query heads of the blocks the tile action
+ * keeps at the query position kv_len[b] - 1 (rit.work TriAttention page, section on
+ * which links may be skipped and which must be kept). Per group g = b * Hkv + kvh:
+ * nkept[g] kept blocks, split into ceil(nkept[g] / bps) items of at most bps blocks
+ * (*blocks_per_split), its first item and partial slot split_start[g]
+ * (split_start[B * Hkv] = *n_items). The kernel hands out every group's splits but
+ * the first (the blocks nearest the diagonal, bps each) first, then the groups' first
+ * splits (block 0 and the far band) in the order first_order lists the groups.
+ * num_sms: the SMs the launch would use (the plan asks for about six items per SM).
+ * Arguments as tria_decode (kv_len, hi, keep host int32); split_start has B * Hkv + 1
+ * entries, first_order and nkept B * Hkv. Returns TRIA_ERR_INVALID_ARG or
+ * TRIA_ERR_UNSUPPORTED as tria_decode would, TRIA_OK otherwise. */
+int tria_decode_plan(int B, int Hq, int Hkv, int T, int capacity, const int32_t* kv_len, const int32_t* hi,
+                     const int32_t* keep, int num_sms, int32_t* split_start, int32_t* first_order, int32_t* nkept,
+                     int32_t* blocks_per_split, int32_t* n_items);
+
 /* Workspace bytes tria_decode needs (0 if the arguments are invalid). */
 size_t tria_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int T, int capacity);
 

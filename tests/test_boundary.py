@@ -18,7 +18,7 @@ def L():
 
 EXPECTED = {
     "tria_status_string", "tria_cache_bytes", "tria_cache_init", "tria_quantize_rows", "tria_quantize_kv",
-    "tria_count_tiles", "tria_prefill_load_plan", "tria_prefill_workspace_bytes", "tria_prefill",
+    "tria_count_tiles", "tria_prefill_load_plan", "tria_decode_plan", "tria_prefill_workspace_bytes", "tria_prefill",
     "tria_prefill_prepare", "tria_prefill_attend", "tria_decode_workspace_bytes", "tria_decode",
     "tria_decode_static", "tria_decode_static_status", "tria_workspace_status",
     "tria_paged_cache_bytes", "tria_paged_cache_init", "tria_cache_status",
