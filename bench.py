@@ -56,11 +56,18 @@ DEFAULT_LEGS = ("decode", "llama_prefill", "llama_prefill_gqa", "long_prefill")
 
 
 def load_peaks():
+    """Measured HBM copy and bf16 GEMM peaks when the measured-peaks file is present and
+    readable (top-level keys hbm_gbs, bf16_tflops, optional bf16_tflops_sustained),
+    else the fallback figures."""
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
-        d = json.loads(p.read_text())
-        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
-                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"])}, "measured"
+        try:
+            d = json.loads(p.read_text())
+            out = {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"])}
+            out["bf16_tflops_sustained"] = float(d.get("bf16_tflops_sustained", out["bf16_tflops"]))
+            return out, "measured"
+        except (ValueError, KeyError, TypeError) as e:
+            print(f"bench: MEASURED_PEAKS.json not usable ({e!r}); fallback peaks", file=sys.stderr)
     return dict(PEAKS_FALLBACK), "fallback"
 
 
