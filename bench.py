@@ -11,9 +11,9 @@ For the decode workload a step is the decode call over a pre-written cache.
 The default workload is the largest single-GPU one: 65,536-token prefill with
 cache write (B1, 32/8 heads, D128, T128). The same run also times, as rows of
 the line, the 64-sequence decode over a 32,768-token compressed cache, the
-8,192-token prefill, the 8,192-token prefill with one policy per KV head (the
-GQA-shared kernel's case) and the two-sequence 32,768-token prefill; `--legs none`
-skips them.
+8,192-token prefill, the 8,192-token and 65,536-token prefills with one policy per KV
+head (the GQA-shared kernel's case) and the two-sequence 32,768-token prefill;
+`--legs none` skips them.
 
 Printed: one JSON line on rank 0. `value` is whole-job throughput with inputs
 resident in HBM; `e2e` times the same calls with the inputs copied from pinned
@@ -52,7 +52,7 @@ from block_sparse_mixed_b200 import workloads as W  # noqa: E402
 L2_FLUSH_BYTES = 256 << 20
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_OVER_BF16 = 2.0   # nominal dense ratio 4.5 POPS int8 / 2.25 PFLOPS bf16: used only if the measurement fails
-DEFAULT_LEGS = ("decode", "llama_prefill", "llama_prefill_gqa", "long_prefill")
+DEFAULT_LEGS = ("decode", "llama_prefill", "llama_prefill_gqa", "long_prefill", "max_prefill_gqa")
 
 
 def load_peaks():

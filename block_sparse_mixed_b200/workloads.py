@@ -54,6 +54,9 @@ WORKLOADS = {
     # (the case the GQA-shared prefill serves)
     "llama_prefill_gqa": Workload("llama_prefill_gqa", "prefill", B=1, Hq=32, Hkv=8, D=128, S=8192,
                                   T=64, seed=6, policy="llama_kv", k_outlier=4.0, k_outlier_frac=0.02),
+    # the 65,536-token shape with the max-context distributions drawn once per KV head
+    "max_prefill_gqa": Workload("max_prefill_gqa", "prefill", B=1, Hq=32, Hkv=8, D=128, S=65536,
+                                T=128, seed=7, policy="maxctx_kv"),
 }
 
 
@@ -71,6 +74,12 @@ def policy(w: Workload) -> tuple[np.ndarray, np.ndarray]:
         for k in range(w.Hkv):
             hi[k * G:(k + 1) * G] = rng.randint(1, 17)
             keep[k * G:(k + 1) * G] = rng.randint(hi[k * G] + 1, 65)
+        return hi, keep
+    if w.policy == "maxctx_kv":        # hi ~ U{2..32}, keep ~ U{hi+8..256} per KV head
+        G = w.Hq // w.Hkv
+        for k in range(w.Hkv):
+            hi[k * G:(k + 1) * G] = rng.randint(2, 33)
+            keep[k * G:(k + 1) * G] = rng.randint(hi[k * G] + 8, 257)
         return hi, keep
     for h in range(w.Hq):
         if w.policy == "llama":        # hi ~ U{1..16}, keep ~ U{hi+1..64}

@@ -70,6 +70,17 @@ def test_long_prefill_full_size_sampled_rows(T, oracle_mod):
     check_rows(oracle_mod, w, Q, K, V, hi, keep, O, L, sampled_picks(w, 96, 1), "long_prefill sampled")
 
 
+def test_max_prefill_gqa_full_size_sampled_rows(T, oracle_mod):
+    """65536 tokens, T = 128, one (hi, keep) per KV head: the GQA-shared kernel at the
+    longest context, on the same sampled rows as the per-head case."""
+    w = W.WORKLOADS["max_prefill_gqa"]
+    hi, keep = W.policy(w)
+    G = w.Hq // w.Hkv
+    assert all(hi[h] == hi[h + 1] and keep[h] == keep[h + 1] for h in range(0, w.Hq, 2)) and G % 2 == 0
+    Q, K, V, hi, keep, _, O, L = run_prefill_like_bench(T, w)
+    check_rows(oracle_mod, w, Q, K, V, hi, keep, O, L, sampled_picks(w, 64, 4), "max_prefill_gqa sampled")
+
+
 def test_max_prefill_full_size_sampled_rows_and_cache(T, oracle_mod):
     """65536 tokens, T = 128; also the compressed cache it writes, bit for bit on sampled tokens."""
     w = W.WORKLOADS["max_prefill"]
