@@ -56,3 +56,18 @@ def test_decode_bytes_count_union_of_planes():
     part8 = 2 * 5 * D + 2 * 5 * 4
     want = full8 + part8 + 2 * full4 + B * Hq * D * 2 + B * Hq * (D * 2 + 4)
     assert bench.decode_bytes(B, Hq, Hkv, D, T, kv, hi, keep) == want
+
+
+def test_peaks_file_read_or_fallback(tmp_path, monkeypatch):
+    """A measured-peaks file with the expected keys is used; one without them (or
+    unreadable) falls back to the fixed figures instead of stopping the run."""
+    import json
+    monkeypatch.setattr(bench, "ROOT", tmp_path)
+    assert bench.load_peaks()[1] == "fallback"
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 7000, "bf16_tflops": 1600}))
+    peaks, src = bench.load_peaks()
+    assert src == "measured" and peaks["hbm_gbs"] == 7000.0 and peaks["bf16_tflops_sustained"] == 1600.0
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm": 1}))
+    assert bench.load_peaks()[1] == "fallback"
+    (tmp_path / "MEASURED_PEAKS.json").write_text("not json")
+    assert bench.load_peaks()[1] == "fallback"
