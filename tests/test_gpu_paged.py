@@ -72,6 +72,8 @@ PREFILL = {
     "D64_T64": (1, 2, 1, 64, 64, 512, 9, [1, 2], [3, 5]),
     # head pairs with equal boundaries: the GQA-shared kernel reads the paged cache
     "D128_T64_gqa_pairs": (2, 4, 2, 128, 64, 640, 12, [2, 2, 0, 0], [5, 5, 9, 9]),
+    "D128_T128_gqa_pairs": (2, 4, 1, 128, 128, 896, 8, [1, 1, 3, 3], [4, 4, 6, 6]),
+    "D64_T128_gqa_pairs": (1, 4, 2, 64, 128, 640, 6, [0, 0, 2, 2], [2, 2, 5, 5]),
 }
 
 
